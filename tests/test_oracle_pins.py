@@ -1,0 +1,476 @@
+"""Pins of the CPU oracle against things other than itself (no GPU needed).
+
+Each test checks the oracle against a closed form, a library routine (numpy /
+scipy), an invariant the definition implies, brute force on tiny inputs, or a
+hand-derived worked example (tests/golden/hand_examples.json).  A plausible
+slip in the oracle -- kmin and kmax swapped, a dropped max(), a sign error, a
+wrong tie-break, an off-by-one forced window, a missing scale, a wrong page
+offset in compaction -- fails at least one of them.
+"""
+
+import dataclasses
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import logsumexp, softmax
+
+import oracle
+import synth
+from synth import Geometry, bf16_to_f32, f32_to_bf16
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")))
+
+
+def _bf(x):
+    return f32_to_bf16(np.asarray(x, dtype=np.float32))
+
+
+def _unpage(case, b, h):
+    """Valid K (and V) tokens of sequence b, KV head h in logical order, as float64."""
+    g = case.geom
+    L = int(case.seq_lens[b])
+    nb = (L + g.P - 1) // g.P
+    ks, vs = [], []
+    for lp in range(nb):
+        ph = case.page_table[b, lp]
+        n = min(g.P, L - lp * g.P)
+        ks.append(case.k_cache[ph, h, :n])
+        if case.v_cache is not None:
+            vs.append(case.v_cache[ph, h, :n])
+        else:
+            vs.append(case.k_cache[ph, h, :n, :g.Dv])
+    k = np.concatenate(ks) if ks else np.zeros((0, g.Dk), np.uint16)
+    v = np.concatenate(vs) if vs else np.zeros((0, g.Dv), np.uint16)
+    return k, v
+
+
+def _f64(bits):
+    return bf16_to_f32(bits).astype(np.float64)
+
+
+# ------------------------------------------------------------------------------------
+# golden worked examples
+# ------------------------------------------------------------------------------------
+
+def test_golden_bound_example():
+    ex = GOLD["bound"]
+    P, D, G = ex["P"], ex["D"], ex["G"]
+    geom = Geometry(B=1, Hq=G, Hkv=1, Dk=D, Dv=D, P=P, max_pages=1, n_pool=1)
+    k = _bf(ex["keys"]).reshape(1, 1, P, D)
+    q = _bf(ex["queries"]).reshape(1, G, D)
+    pt = np.zeros((1, 1), np.int32)
+    sl = np.array([P], np.int32)
+    summ = oracle.page_summaries(geom, k, pt, sl)
+    assert np.array_equal(_f64(summ[0, 0, 0]), ex["kmin"])
+    assert np.array_equal(_f64(summ[0, 0, 1]), ex["kmax"])
+    sc = oracle.page_scores(geom, q, summ, pt, sl)
+    assert sc[0, 0, 0] == ex["score"]
+    assert ex["true_max_qk"] <= sc[0, 0, 0]
+
+
+def test_golden_select_examples():
+    ex = GOLD["select"]
+    for c in ex["cases"]:
+        n = len(c["scores"])
+        geom = Geometry(B=1, Hq=1, Hkv=1, Dk=8, Dv=8, P=ex["P"], max_pages=n, n_pool=n)
+        sc = np.asarray(c["scores"], np.float64).reshape(1, 1, n)
+        sel, cnt = oracle.select_pages(geom, sc, np.array([n * ex["P"]], np.int32),
+                                       ex["budget"], ex["sink"], ex["window"])
+        assert cnt[0, 0] == len(c["sel"])
+        assert list(sel[0, 0, :cnt[0, 0]]) == c["sel"], c["derivation"]
+        assert (sel[0, 0, cnt[0, 0]:] == -1).all()
+
+
+def test_golden_attend_example():
+    ex = GOLD["attend"]
+    q = _bf([ex["q"]])
+    out, lse = oracle.dense_attend(q, _bf(ex["keys"]), _bf(ex["values"]), ex["scale"])
+    assert np.allclose(out[0], ex["out"], rtol=0, atol=1e-15)
+    assert abs(lse[0] - ex["lse"]) < 1e-15
+    # closed forms
+    e = math.e
+    assert abs(out[0, 0] - 1 / (1 + e)) < 1e-15 and abs(lse[0] - math.log1p(e)) < 1e-15
+
+
+def test_golden_prune_example():
+    ex = GOLD["prune"]
+    P, L = ex["P"], ex["L"]
+    n_pool = 8
+    geom = Geometry(B=1, Hq=1, Hkv=1, Dk=8, Dv=8, P=P, max_pages=3, n_pool=n_pool)
+    k = np.arange(n_pool * P * 8, dtype=np.uint16).reshape(n_pool, 1, P, 8) + 0x3F00
+    v = k + 7
+    pt = np.array([[0, 1, 2]], np.int32)
+    keep = np.zeros((1, 3 * P), np.uint8)
+    keep[0, :L] = ex["keep"]
+    r = oracle.prune_compact(geom, k, v, pt, np.array([L], np.int32), keep,
+                             np.asarray(ex["free_pages"], np.int32))
+    assert r["new_seq_lens"][0] == ex["new_seq_len"]
+    assert list(r["new_page_table"][0, :2]) == ex["new_pages"] and r["new_page_table"][0, 2] == -1
+    assert list(r["pos_map"][0, :3]) == ex["pos_map"] and (r["pos_map"][0, 3:] == -1).all()
+    assert r["logical_len"][0] == ex["logical_len"]
+    # slot contents: token t of the source lives in page t // P, slot t % P
+    for i, t in enumerate(ex["pos_map"]):
+        dst = ex["new_pages"][i // P]
+        assert np.array_equal(r["k_dst"][dst, 0, i % P], k[t // P, 0, t % P])
+        assert np.array_equal(r["v_dst"][dst, 0, i % P], v[t // P, 0, t % P])
+    assert (r["k_dst"][4, 0, 1] == 0).all() and (r["v_dst"][4, 0, 1] == 0).all()
+
+
+# ------------------------------------------------------------------------------------
+# (1) summaries
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("P,lens", [(16, [0, 1, 15, 16, 17, 100]), (32, [31, 33, 64]),
+                                    (64, [1, 63, 65, 200])])
+def test_summaries_match_numpy_min_max(P, lens):
+    case = synth.decode_case("tiny", B=len(lens), seq_lens=lens, P=P, Hkv=2, Hq=4,
+                             identity=False, extra_pool_pages=5, poison="nan")
+    g = case.geom
+    summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    for b, L in enumerate(lens):
+        for lp in range((L + P - 1) // P):
+            ph = case.page_table[b, lp]
+            n = min(P, L - lp * P)
+            for h in range(g.Hkv):
+                x = bf16_to_f32(case.k_cache[ph, h, :n])      # valid tokens only
+                assert np.array_equal(bf16_to_f32(summ[ph, h, 0]), x.min(axis=0))
+                assert np.array_equal(bf16_to_f32(summ[ph, h, 1]), x.max(axis=0))
+    # pages nobody references stay untouched
+    used = set(case.page_table[case.page_table >= 0].tolist())
+    for ph in range(g.n_pool):
+        if ph not in used:
+            assert (summ[ph] == 0).all()
+
+
+def test_summaries_signed_zero_and_single_token():
+    geom = Geometry(B=1, Hq=1, Hkv=1, Dk=4, Dv=4, P=16, max_pages=1, n_pool=1)
+    k = np.zeros((1, 1, 16, 4), np.uint16)
+    k[0, 0, 0] = [0x8000, 0x0000, 0x3F80, 0xBF80]   # -0, +0, 1, -1
+    k[0, 0, 1] = [0x0000, 0x8000, 0x3F80, 0xBF80]
+    summ = oracle.page_summaries(geom, k, np.zeros((1, 1), np.int32), np.array([2], np.int32))
+    assert list(summ[0, 0, 0]) == [0x8000, 0x8000, 0x3F80, 0xBF80]
+    assert list(summ[0, 0, 1]) == [0x0000, 0x0000, 0x3F80, 0xBF80]
+    # one valid token: min == max == that token (bitwise)
+    summ1 = oracle.page_summaries(geom, k, np.zeros((1, 1), np.int32), np.array([1], np.int32))
+    assert np.array_equal(summ1[0, 0, 0], k[0, 0, 0]) and np.array_equal(summ1[0, 0, 1], k[0, 0, 0])
+
+
+# ------------------------------------------------------------------------------------
+# (2) page scores
+# ------------------------------------------------------------------------------------
+
+def _small_case(**kw):
+    base = dict(B=2, seq_lens=[300, 517], Hq=8, Hkv=2, identity=False, extra_pool_pages=3)
+    base.update(kw)
+    return synth.decode_case("tiny", **base)
+
+
+def test_bound_dominates_true_max_qk():
+    case = _small_case()
+    g = case.geom
+    summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    sc = oracle.page_scores(g, case.q, summ, case.page_table, case.seq_lens)
+    qf = _f64(case.q)
+    for b in range(g.B):
+        L = int(case.seq_lens[b])
+        for h in range(g.Hkv):
+            k, _ = _unpage(case, b, h)
+            qk = qf[b, h * g.G:(h + 1) * g.G] @ _f64(k).T          # [G, L]
+            for lp in range((L + g.P - 1) // g.P):
+                true_max = qk[:, lp * g.P:min(L, (lp + 1) * g.P)].max()
+                assert sc[b, h, lp] >= true_max - 1e-12
+        assert np.isneginf(sc[b, :, (L + g.P - 1) // g.P:]).all()
+
+
+def test_bound_equals_qk_for_single_token_pages():
+    # P = 1 (forced through a one-token-per-page case) and G = 1: bound == q.k exactly
+    geom = Geometry(B=1, Hq=1, Hkv=1, Dk=64, Dv=64, P=1, max_pages=50, n_pool=50)
+    rng = np.random.default_rng(0)
+    k = _bf(rng.standard_normal((50, 1, 1, 64)))
+    q = _bf(rng.standard_normal((1, 1, 64)))
+    pt = rng.permutation(50).astype(np.int32).reshape(1, 50)
+    sl = np.array([50], np.int32)
+    summ = oracle.page_summaries(geom, k, pt, sl)
+    sc = oracle.page_scores(geom, q, summ, pt, sl)
+    expect = _f64(k[pt[0], 0, 0]) @ _f64(q[0, 0])
+    assert np.array_equal(sc[0, 0], expect) or np.allclose(sc[0, 0], expect, rtol=0, atol=1e-12)
+
+
+def test_bound_split_sign_identity():
+    # max(q*kmax, q*kmin) == max(q,0)*kmax + min(q,0)*kmin because kmax >= kmin;
+    # evaluated here with a library matmul, then the GQA max-reduction.
+    case = _small_case(Hq=16, Hkv=2)
+    g = case.geom
+    summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    sc = oracle.page_scores(g, case.q, summ, case.page_table, case.seq_lens)
+    qf = _f64(case.q)
+    for b in range(g.B):
+        nb = (int(case.seq_lens[b]) + g.P - 1) // g.P
+        phys = case.page_table[b, :nb]
+        for h in range(g.Hkv):
+            kmin = _f64(summ[phys, h, 0])      # [nb, D]
+            kmax = _f64(summ[phys, h, 1])
+            qg = qf[b, h * g.G:(h + 1) * g.G]   # [G, D]
+            u = np.maximum(qg, 0) @ kmax.T + np.minimum(qg, 0) @ kmin.T
+            assert np.allclose(sc[b, h, :nb], u.max(axis=0), rtol=1e-13, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------
+# (3) selection
+# ------------------------------------------------------------------------------------
+
+def _brute_select(scores, n, K, s, w):
+    """The unique set in which every chosen candidate beats every unchosen one."""
+    if n <= K:
+        return list(range(n))
+    forced = [p for p in range(n) if p < s or p >= n - w]
+    cands = [p for p in range(n) if p not in forced]
+    k_top = K - s - w
+    better = lambda a, b: scores[a] > scores[b] or (scores[a] == scores[b] and a < b)
+    found = []
+    for sub in itertools.combinations(cands, k_top):
+        rest = [p for p in cands if p not in sub]
+        if all(better(a, r) for a in sub for r in rest):
+            found.append(sub)
+    assert len(found) == 1
+    return sorted(forced + list(found[0]))
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_select_brute_force_tiny(seed):
+    rng = np.random.default_rng(seed)
+    P = 16
+    n = int(rng.integers(1, 13))
+    K = int(rng.integers(2, 9))
+    s = int(rng.integers(0, K + 1))
+    w = int(rng.integers(0, K - s + 1))
+    # few distinct values -> many ties
+    scores = rng.integers(-3, 4, size=n).astype(np.float64) * 0.5
+    geom = Geometry(B=1, Hq=1, Hkv=1, Dk=8, Dv=8, P=P, max_pages=n, n_pool=n)
+    sel, cnt = oracle.select_pages(geom, scores.reshape(1, 1, n), np.array([n * P - 3], np.int32),
+                                   K * P, s * P, w * P)
+    want = _brute_select(scores, n, K, s, w)
+    assert list(sel[0, 0, :cnt[0, 0]]) == want
+
+
+def test_select_forced_pages_and_counts():
+    case = synth.decode_case("tiny", B=3, seq_lens=[4096, 700, 50], Hkv=2, Hq=8)
+    g = case.geom
+    r = oracle.decode(case)
+    K, s, w = case.budget // g.P, case.sink // g.P, case.window // g.P
+    for b in range(g.B):
+        nb = (int(case.seq_lens[b]) + g.P - 1) // g.P
+        for h in range(g.Hkv):
+            c = int(r["sel_count"][b, h])
+            sel = list(r["sel"][b, h, :c])
+            assert c == min(nb, K)
+            assert sel == sorted(set(sel))
+            if nb > K:
+                assert set(range(s)) <= set(sel)
+                assert set(range(nb - w, nb)) <= set(sel)
+
+
+def test_select_matches_library_lexsort():
+    case = synth.decode_case("llama32k", B=2, L=(8192, 8192), seed=7)
+    g = case.geom
+    r = oracle.decode(case)
+    K, s, w = case.budget // g.P, case.sink // g.P, case.window // g.P
+    for b in range(g.B):
+        nb = g.max_pages
+        for h in range(g.Hkv):
+            sc = r["scores"][b, h, :nb]
+            cand = np.arange(s, nb - w)
+            order = np.lexsort((cand, -sc[cand]))     # score desc, index asc
+            want = np.sort(np.concatenate([np.arange(s), cand[order[:K - s - w]],
+                                           np.arange(nb - w, nb)]))
+            assert np.array_equal(r["sel"][b, h], want)
+
+
+def test_selection_invariant_under_page_permutation():
+    case = synth.decode_case("tiny", B=2, seq_lens=[1000, 3000], Hkv=2, Hq=8, identity=True)
+    r1 = oracle.decode(case)
+    g = case.geom
+    perm = np.random.default_rng(3).permutation(g.n_pool)        # old phys -> new phys
+    k2 = np.empty_like(case.k_cache)
+    v2 = np.empty_like(case.v_cache)
+    k2[perm] = case.k_cache
+    v2[perm] = case.v_cache
+    pt2 = np.where(case.page_table >= 0, perm[np.maximum(case.page_table, 0)], -1).astype(np.int32)
+    case2 = dataclasses.replace(case, k_cache=k2, v_cache=v2, page_table=pt2)
+    r2 = oracle.decode(case2)
+    assert np.array_equal(r1["sel"], r2["sel"]) and np.array_equal(r1["sel_count"], r2["sel_count"])
+    assert np.array_equal(r1["out"], r2["out"]) and np.array_equal(r1["lse"], r2["lse"])
+
+
+# ------------------------------------------------------------------------------------
+# (4) attention
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wl", ["tiny", "mla"])
+def test_full_budget_equals_dense_attention(wl):
+    if wl == "tiny":
+        case = synth.decode_case("tiny", B=2, seq_lens=[777, 1024], Hkv=2, Hq=8, budget=1024,
+                                 poison="nan")
+    else:
+        case = synth.decode_case("mla", B=1, seq_lens=[300], Hq=8, budget=384, sink=64,
+                                 window=128, poison="nan")
+    g = case.geom
+    r = oracle.decode(case)
+    for b in range(g.B):
+        assert r["sel_count"][b].min() == (int(case.seq_lens[b]) + g.P - 1) // g.P
+        for h in range(g.Hkv):
+            k, v = _unpage(case, b, h)
+            qg = case.q[b, h * g.G:(h + 1) * g.G]
+            out_d, lse_d = oracle.dense_attend(qg, k, v, case.scale)
+            sl = slice(h * g.G, (h + 1) * g.G)
+            assert np.allclose(r["out"][b, sl], out_d, rtol=0, atol=1e-12)
+            assert np.allclose(r["lse"][b, sl], lse_d, rtol=0, atol=1e-12)
+            # textbook form with library routines
+            x = case.scale * (_f64(qg) @ _f64(k).T)
+            assert np.allclose(out_d, softmax(x, axis=1) @ _f64(v), rtol=0, atol=1e-12)
+            assert np.allclose(lse_d, logsumexp(x, axis=1), rtol=0, atol=1e-12)
+
+
+def test_attend_single_token_and_uniform_logits():
+    geom = Geometry(B=2, Hq=2, Hkv=1, Dk=64, Dv=64, P=16, max_pages=4, n_pool=8)
+    rng = np.random.default_rng(5)
+    k = _bf(rng.standard_normal((8, 1, 16, 64)))
+    v = _bf(rng.standard_normal((8, 1, 16, 64)))
+    q = _bf(rng.standard_normal((2, 2, 64)))
+    q[1] = 0                                               # uniform logits for sequence 1
+    pt = np.array([[5, -1, -1, -1], [2, 6, 1, 3]], np.int32)
+    sl = np.array([1, 50], np.int32)
+    sel = np.array([[[0, -1, -1, -1]], [[0, 1, 2, 3]]], np.int32)
+    cnt = np.array([[1], [4]], np.int32)
+    out, lse = oracle.attend(geom, q, k, v, pt, sl, sel, cnt, 0.125)
+    # one token: o = v, lse = scale * q.k
+    assert np.array_equal(out[0, 0], _f64(v[5, 0, 0])) and np.array_equal(out[0, 1], _f64(v[5, 0, 0]))
+    assert np.allclose(lse[0], 0.125 * (_f64(q[0]) @ _f64(k[5, 0, 0])), rtol=0, atol=1e-12)
+    # q = 0: every logit is 0 -> o = mean of the 50 valid values, lse = log 50
+    vv = np.concatenate([_f64(v[2, 0]), _f64(v[6, 0]), _f64(v[1, 0]), _f64(v[3, 0, :2])])
+    assert np.allclose(out[1, 0], vv.mean(axis=0), rtol=0, atol=1e-12)
+    assert np.allclose(lse[1], math.log(50), rtol=0, atol=1e-12)
+
+
+def test_attend_empty_sequence():
+    case = synth.decode_case("tiny", B=2, seq_lens=[0, 40], Hkv=1, Hq=4)
+    r = oracle.decode(case)
+    assert r["sel_count"][0, 0] == 0 and (r["sel"][0, 0] == -1).all()
+    assert (r["out"][0] == 0).all() and np.isneginf(r["lse"][0]).all()
+
+
+def test_attend_matches_numpy_on_sparse_selection():
+    case = synth.decode_case("llama32k", B=1, L=(4096, 4096), seed=11, poison="inf")
+    g = case.geom
+    r = oracle.decode(case)
+    for h in range(g.Hkv):
+        k, v = _unpage(case, 0, h)
+        cnt = r["sel_count"][0, h]
+        toks = np.concatenate([np.arange(p * g.P, (p + 1) * g.P) for p in r["sel"][0, h, :cnt]])
+        qg = _f64(case.q[0, h * g.G:(h + 1) * g.G])
+        x = case.scale * (qg @ _f64(k[toks]).T)
+        sl = slice(h * g.G, (h + 1) * g.G)
+        assert np.allclose(r["out"][0, sl], softmax(x, axis=1) @ _f64(v[toks]), rtol=0, atol=1e-12)
+        assert np.allclose(r["lse"][0, sl], logsumexp(x, axis=1), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------
+# (5) prefix-cache pruning
+# ------------------------------------------------------------------------------------
+
+def _small_prune(**kw):
+    base = dict(B=3, seq_lens=[3000, 2200, 5000], Hkv=2, Hq=8, P=16)
+    base.update(kw)
+    return synth.prune_case("prune", **base)
+
+
+def test_prune_round_trip_and_allocation_rule():
+    pc = _small_prune(extra_free=4)
+    d = pc.decode
+    g = d.geom
+    r = oracle.prune_compact(g, d.k_cache, d.v_cache, d.page_table, d.seq_lens, pc.keep,
+                             pc.free_pages)
+    off = 0
+    width = g.max_pages * g.P
+    for b in range(g.B):
+        L = int(d.seq_lens[b])
+        kept_pos = np.nonzero(pc.keep[b, :L])[0]
+        Lp = len(kept_pos)
+        assert r["new_seq_lens"][b] == Lp and r["logical_len"][b] == L
+        assert np.array_equal(r["pos_map"][b, :Lp], kept_pos)
+        assert (r["pos_map"][b, Lp:width] == -1).all()
+        npg = (Lp + g.P - 1) // g.P
+        assert np.array_equal(r["new_page_table"][b, :npg], pc.free_pages[off:off + npg])
+        assert (r["new_page_table"][b, npg:] == -1).all()
+        # expand(compact(x)) == x on the kept positions
+        for h in range(g.Hkv):
+            kc = np.concatenate([r["k_dst"][p, h] for p in r["new_page_table"][b, :npg]])[:Lp]
+            vc = np.concatenate([r["v_dst"][p, h] for p in r["new_page_table"][b, :npg]])[:Lp]
+            k0, v0 = _unpage(d, b, h)
+            assert np.array_equal(kc, k0[kept_pos]) and np.array_equal(vc, v0[kept_pos])
+            # summaries of the new pages == numpy min/max of the compacted tokens
+            for j in range(npg):
+                x = bf16_to_f32(kc[j * g.P:(j + 1) * g.P])
+                p = r["new_page_table"][b, j]
+                assert np.array_equal(bf16_to_f32(r["summ"][p, h, 0]), x.min(axis=0))
+                assert np.array_equal(bf16_to_f32(r["summ"][p, h, 1]), x.max(axis=0))
+        off += npg
+    assert r["pages_used"] == off
+    # the old pages were not modified
+    assert np.array_equal(r["k_dst"][d.page_table[d.page_table >= 0]],
+                          d.k_cache[d.page_table[d.page_table >= 0]])
+
+
+def test_prune_keep_all_and_keep_none():
+    pa = _small_prune(keep_all=True)
+    d = pa.decode
+    g = d.geom
+    ra = oracle.prune_compact(g, d.k_cache, d.v_cache, d.page_table, d.seq_lens, pa.keep,
+                              pa.free_pages)
+    assert np.array_equal(ra["new_seq_lens"], d.seq_lens)
+    for b in range(g.B):
+        for h in range(g.Hkv):
+            k0, _ = _unpage(d, b, h)
+            npg = (int(d.seq_lens[b]) + g.P - 1) // g.P
+            kc = np.concatenate([ra["k_dst"][p, h] for p in ra["new_page_table"][b, :npg]])
+            assert np.array_equal(kc[:len(k0)], k0)
+    pn = _small_prune(keep_none=True)
+    d = pn.decode
+    rn = oracle.prune_compact(d.geom, d.k_cache, d.v_cache, d.page_table, d.seq_lens, pn.keep,
+                              pn.free_pages)
+    assert rn["pages_used"] == 0 and (rn["new_seq_lens"] == 0).all()
+    assert (rn["new_page_table"] == -1).all() and (rn["pos_map"] == -1).all()
+    assert np.array_equal(rn["logical_len"], d.seq_lens)
+
+
+def test_prune_not_enough_free_pages():
+    pc = _small_prune()
+    d = pc.decode
+    with pytest.raises(ValueError):
+        oracle.prune_compact(d.geom, d.k_cache, d.v_cache, d.page_table, d.seq_lens, pc.keep,
+                             pc.free_pages[:-1])
+
+
+def test_decode_after_prune_full_budget_equals_dense_on_kept_tokens():
+    pc = _small_prune(extra_free=0)
+    d = pc.decode
+    g = d.geom
+    r = oracle.prune_compact(g, d.k_cache, d.v_cache, d.page_table, d.seq_lens, pc.keep,
+                             pc.free_pages)
+    big = g.max_pages * g.P
+    sc = oracle.page_scores(g, d.q, r["summ"], r["new_page_table"], r["new_seq_lens"])
+    sel, cnt = oracle.select_pages(g, sc, r["new_seq_lens"], big, 0, 0)
+    out, lse = oracle.attend(g, d.q, r["k_dst"], r["v_dst"], r["new_page_table"],
+                             r["new_seq_lens"], sel, cnt, d.scale)
+    for b in range(g.B):
+        keptpos = r["pos_map"][b, :r["new_seq_lens"][b]]
+        for h in range(g.Hkv):
+            k0, v0 = _unpage(d, b, h)
+            od, ld = oracle.dense_attend(d.q[b, h * g.G:(h + 1) * g.G], k0[keptpos], v0[keptpos],
+                                         d.scale)
+            assert np.allclose(out[b, h * g.G:(h + 1) * g.G], od, rtol=0, atol=1e-12)
+            assert np.allclose(lse[b, h * g.G:(h + 1) * g.G], ld, rtol=0, atol=1e-12)
