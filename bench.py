@@ -1,0 +1,485 @@
+"""Throughput of query-aware page-sparse decode over a paged KV cache on B200.
+
+One step = one decode step of a 32-layer model with Llama-3.1-8B attention geometry
+(batch 8, 32 query / 8 KV heads, head dim 128, 32768 tokens per sequence, page 16,
+token budget 2048 = sink 64 + window 512 + top-k): for every layer, the summary of
+each sequence's newest page is refreshed (sa_update_summaries), every page is scored
+and the top pages selected (sa_select_pages: scoring + top-k kernels), and attention
+runs over the gathered pages (sa_attend_selected: split-KV attention + merge) -- the
+two halves of sa_sparse_decode, called separately so the bench can time each.
+Every layer owns its own KV pool, so a step touches ~4.3 GB (> L2) and nothing is
+served from L2 across layers.
+
+Metric: sparse-decode seq*heads/s = (sequence, query head) attention outputs of one
+layer-call per second, whole job.  Also printed: achieved HBM GB/s of the whole step
+and, in "roofline", of the dominant kernel, against MEASURED_PEAKS.json.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama32k|llama128k|ragged]
+  python bench.py --impl reference ...   (the CPU oracle on a bounded sample)
+
+Under torchrun (N > 1) every rank runs its own batch on its own GPU (weak scaling,
+no collective on the data path); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+N_LAYERS = 32
+WORKLOADS = ("llama32k", "llama128k", "ragged")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama32k", choices=WORKLOADS)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layer pools per step (default 32 for llama32k, 8 otherwise)")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-parity", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def _json_default(o):
+    if hasattr(o, "item"):
+        return o.item()
+    return str(o)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------
+# algorithmic bytes (inherent to the method; workspace traffic excluded)
+# ------------------------------------------------------------------------------------
+
+def layer_bytes(geom, seq_lens, sel_count, P):
+    """Per layer-call: (select_bytes, attend_bytes, update_bytes)."""
+    g = geom
+    nb = (seq_lens.astype(np.int64) + P - 1) // P
+    summ = int(nb.sum()) * g.Hkv * 2 * g.Dk * 2
+    pt = int(nb.sum()) * 4
+    q = g.B * g.Hq * g.Dk * 2
+    sel_bytes = summ + pt + q
+    # valid tokens of the selected pages: every selected page is full except a
+    # sequence's last page (always selected when the sequence is non-empty)
+    tok = 0
+    for b in range(g.B):
+        L = int(seq_lens[b])
+        last_valid = L - (nb[b] - 1) * P if nb[b] else 0
+        for h in range(g.Hkv):
+            c = int(sel_count[b, h])
+            tok += c * P - (P - last_valid if c else 0)
+    kv = tok * (g.Dk + (0 if g.v_aliases_k else g.Dv)) * 2
+    att_bytes = kv + q + g.B * g.Hq * (g.Dv * 4 + 4)
+    upd = g.B * g.Hkv * (P * g.Dk * 2 + 2 * g.Dk * 2)
+    return sel_bytes, att_bytes, upd
+
+
+# ------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------
+# CPU oracle arm (cpu_baseline and --impl reference)
+# ------------------------------------------------------------------------------------
+
+def oracle_sample(case, seconds):
+    """Time the CPU oracle's decode step (score + select + attend) sequence by sequence
+    on the bench's own layer-0 data until ~`seconds` have elapsed."""
+    import oracle
+    g = case.geom
+    summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    done, t_total = 0, 0.0
+    b = 0
+    while t_total < seconds:
+        sub = synth.Geometry(1, g.Hq, g.Hkv, g.Dk, g.Dv, g.P, g.max_pages, g.n_pool, g.v_aliases_k)
+        q = case.q[b:b + 1]
+        pt = case.page_table[b:b + 1]
+        sl = case.seq_lens[b:b + 1]
+        t0 = time.perf_counter()
+        sc = oracle.page_scores(sub, q, summ, pt, sl)
+        sel, cnt = oracle.select_pages(sub, sc, sl, case.budget, case.sink, case.window)
+        oracle.attend(sub, q, case.k_cache, case.v_cache, pt, sl, sel, cnt, case.scale)
+        t_total += time.perf_counter() - t0
+        done += 1
+        b = (b + 1) % g.B
+    units = done * g.Hq
+    return units / t_total, done, t_total
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    case = synth.decode_case(args.workload)
+    v, done, t = oracle_sample(case, args.cpu_seconds)
+    line = {
+        "impl": "reference", "metric": "sparse-decode seq*heads/s", "value": v,
+        "unit": "seq*heads/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "ms_per_step": None,
+        "config": {"workload": args.workload, "layers_per_step": args.layers},
+        "cpu_baseline": {"value": v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
+                         "sample": "%d (sequence, layer) decode calls of layer 0 "
+                                   "(score+select+attend, all %d heads), %.1f s" % (
+                                       done, case.geom.Hq, t)},
+        "e2e": {"value": v, "unit": "seq*heads/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line, default=_json_default), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------
+# native arm
+# ------------------------------------------------------------------------------------
+
+def run_native(args, rank, world, dist):
+    import torch
+    import paged_kv_cache_sa_b200 as sa
+    from paged_kv_cache_sa_b200 import Geometry
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    hbm_peak, _, peak_kind = peaks()
+
+    # ---- inputs: layer 0 from the seeded generator (rank-specific seed), other layers
+    # are the same bytes rolled along the page axis (distinct memory and content)
+    case = synth.decode_case(args.workload, seed=synth.WORKLOADS[args.workload]["seed"] + 1000 * rank)
+    g = Geometry.of(case.geom)
+    P = g.P
+    L_layers = args.layers
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16
+                                                          else a)).to(dev)
+    k0, v0 = t(case.k_cache), t(case.v_cache)
+    pt, sl = t(case.page_table), t(case.seq_lens)
+    rng = np.random.default_rng(1234 + rank)
+    ks, vs, qs, summs = [], [], [], []
+    stride = max(1, g.n_pool // L_layers)
+    for l in range(L_layers):
+        ks.append(k0 if l == 0 else torch.roll(k0, shifts=l * stride, dims=0))
+        vs.append(v0 if l == 0 else torch.roll(v0, shifts=l * stride, dims=0))
+        qn = case.q if l == 0 else synth.f32_to_bf16(rng.standard_normal(case.q.shape).astype(np.float32))
+        qs.append(t(qn))
+        summs.append(torch.empty((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device=dev))
+        sa.page_summaries(g, ks[l], pt, sl, summs[l])
+    K = case.budget // P
+    ws = sa.Workspace.for_decode(g, case.budget)
+    sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((g.B, g.Hkv), dtype=torch.int32, device=dev)
+    outs = [torch.empty((g.B, g.Hq, g.Dv), dtype=torch.float32, device=dev) for _ in range(L_layers)]
+    lses = [torch.empty((g.B, g.Hq), dtype=torch.float32, device=dev) for _ in range(L_layers)]
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+          for _ in range(L_layers)]
+
+    def step(with_events):
+        for l in range(L_layers):
+            if with_events:
+                ev[l][0].record()
+            sa.update_summaries(g, ks[l], pt, sl, summs[l], 1)
+            sa.select_pages(g, qs[l], summs[l], pt, sl, case.budget, case.sink, case.window, ws,
+                            sel=sel, sel_count=cnt)
+            if with_events:
+                ev[l][1].record()
+            sa.attend_selected(g, qs[l], ks[l], vs[l], pt, sl, sel, cnt, case.scale, ws,
+                               out=outs[l], lse=lses[l])
+            if with_events:
+                ev[l][2].record()
+
+    # one eager step: correctness of the launch config, selection counts for the bytes
+    step(False)
+    assert ws.status() == sa.SA_OK
+    sel_count = cnt.cpu().numpy()
+    sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, P)
+    step_bytes = L_layers * (sel_b + att_b + upd_b)
+
+    # capture one step (with per-layer events) in a CUDA graph
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        step(True)                      # warm the stream before capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            step(True)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t0e = torch.cuda.Event(enable_timing=True)
+    t1e = torch.cuda.Event(enable_timing=True)
+    sel_ms = np.zeros(L_layers)
+    att_ms = np.zeros(L_layers)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0e.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        t1e.record(stream)
+    torch.cuda.synchronize()
+    total_ms = t0e.elapsed_time(t1e)
+    # per-phase durations: events of the last replay (identical work every replay)
+    for l in range(L_layers):
+        sel_ms[l] = ev[l][0].elapsed_time(ev[l][1])
+        att_ms[l] = ev[l][1].elapsed_time(ev[l][2])
+    clk = clocks.stop()
+    if dist is not None:
+        import torch.distributed as tdist
+        tt = torch.tensor([total_ms], device=dev)
+        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    units_per_step = g.B * g.Hq * L_layers
+    value = units_per_step * world / (ms_per_step * 1e-3)
+    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # ---- e2e through the public API with host buffers: q H2D + out/lse D2H every step
+    q_host = [torch.empty(qs[l].shape, dtype=torch.int16).pin_memory() for l in range(L_layers)]
+    for l in range(L_layers):
+        q_host[l].copy_(qs[l].cpu())
+    o_host = [torch.empty(outs[l].shape, dtype=torch.float32).pin_memory() for l in range(L_layers)]
+    l_host = [torch.empty(lses[l].shape, dtype=torch.float32).pin_memory() for l in range(L_layers)]
+    e2e_steps = max(3, args.steps // 2)
+    with torch.cuda.stream(stream):
+        for it in range(e2e_steps + 2):
+            if it == 2:
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            for l in range(L_layers):
+                qs[l].copy_(q_host[l], non_blocking=True)
+            graph.replay()
+            for l in range(L_layers):
+                o_host[l].copy_(outs[l], non_blocking=True)
+                l_host[l].copy_(lses[l], non_blocking=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist is not None:
+        import torch.distributed as tdist
+        tt = torch.tensor([e2e_ms], device=dev)
+        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = sum(int(x.numel()) * 2 for x in q_host)
+    d2h = sum(int(x.numel()) * 4 for x in o_host) + sum(int(x.numel()) * 4 for x in l_host)
+
+    # ---- sampled parity at full size: layer 0 against the oracle
+    parity = None
+    if rank == 0 and not args.no_parity:
+        parity = full_size_parity(case, outs[0], lses[0], sel, cnt, sa, g, ks, vs, qs, summs, pt,
+                                  sl, ws, dev)
+
+    if rank != 0:
+        return 0
+    att_mean = float(att_ms.mean())
+    sel_mean = float(sel_ms.mean())
+    dom_is_att = att_mean >= sel_mean
+    dom_ms = att_mean if dom_is_att else sel_mean
+    dom_bytes = att_b if dom_is_att else sel_b
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    cpu_v, cpu_done, cpu_t = (None, 0, 0.0)
+    if world == 1:
+        cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    launches_per_layer = 4 + (1 if plan_nsplit(g, case.budget, sms) > 1 else 0)
+    line = {
+        "metric": "sparse-decode seq*heads/s",
+        "value": value,
+        "unit": "seq*heads/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": args.workload,
+            "batch": g.B, "q_heads": g.Hq, "kv_heads": g.Hkv, "head_dim": g.Dk,
+            "seq_len": int(case.seq_lens.max()), "page": P, "budget_tokens": case.budget,
+            "sink": case.sink, "window": case.window, "layers_per_step": L_layers,
+            "l2": "inputs larger than L2: %d distinct layer pools, %.2f GB touched per step"
+                  % (L_layers, step_bytes / 1e9),
+            "parallelism": "replicas (batch split), no collective" if world > 1 else "1 GPU",
+            "step_hbm_gbs": step_gbs,
+            "step_frac_of_hbm_peak": step_gbs / hbm_peak,
+            "select_us_per_layer": sel_mean * 1e3,
+            "attend_us_per_layer": att_mean * 1e3,
+            "algorithmic_bytes_per_layer": sel_b + att_b + upd_b,
+        },
+        "roofline": {
+            "kernel": "attend_gqa_kernel+merge_kernel" if dom_is_att
+            else "update+score_gqa_kernel+topk_kernel",
+            "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "peak_kind": peak_kind + " (burst copy)",
+            "traffic": None,
+        },
+        "cpu_baseline": None if cpu_v is None else {
+            "value": cpu_v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
+            "sample": "%d (sequence, layer) decode calls of layer 0 (score+select+attend over "
+                      "all %d query heads), %.1f s single-threaded" % (cpu_done, g.Hq, cpu_t)},
+        "e2e": {"value": units_per_step * world / (e2e_ms * 1e-3), "unit": "seq*heads/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_layer * L_layers * args.steps,
+        "clocks": clk,
+        "parity": parity,
+    }
+    print(json.dumps(line, default=_json_default), flush=True)
+    return 0
+
+
+def plan_nsplit(g, budget, sm_count):
+    """Attention CTAs per (sequence, KV head) as the library plans them (same rule)."""
+    K = budget // g.P
+    units = g.B * g.Hkv
+    ns = max(1, min(K, (4 * sm_count + units - 1) // units))
+    pps = min(256, (((K + ns - 1) // ns) + 3) & ~3)
+    return (K + pps - 1) // pps
+
+
+def full_size_parity(case, out0, lse0, sel, cnt, sa, g, ks, vs, qs, summs, pt, sl, ws, dev):
+    """Layer 0 at full size, in the bench's launch configuration, against the oracle:
+    selection bit-exact (tie band aside) and attention within tolerance for every
+    sequence and head."""
+    import torch
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity import check_attention, check_selection
+    sa.select_pages(g, qs[0], summs[0], pt, sl, case.budget, case.sink, case.window, ws,
+                    sel=sel, sel_count=cnt)
+    sa.attend_selected(g, qs[0], ks[0], vs[0], pt, sl, sel, cnt, case.scale, ws, out=out0,
+                       lse=lse0)
+    torch.cuda.synchronize()
+    gs, gc = sel.cpu().numpy(), cnt.cpu().numpy()
+    summ = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    gsumm = summs[0].cpu().numpy().view(np.uint16)
+    summ_ok = bool(np.array_equal(gsumm, summ))
+    sc = oracle.page_scores(case.geom, case.q, summ, case.page_table, case.seq_lens)
+    osel, ocnt = oracle.select_pages(case.geom, sc, case.seq_lens, case.budget, case.sink,
+                                     case.window)
+    tied = check_selection(case.geom, case.seq_lens, case.budget, case.sink, case.window, sc,
+                           osel, ocnt, gs, gc)
+    o, l = oracle.attend(case.geom, case.q, case.k_cache, case.v_cache, case.page_table,
+                         case.seq_lens, gs if tied else osel, ocnt, case.scale)
+    err, rel, lerr = check_attention(out0.cpu().numpy(), lse0.cpu().numpy(), o, l)
+    return {"layer": 0, "summaries_bit_exact": summ_ok, "selection_bit_exact": not tied,
+            "tie_band_units": len(tied), "out_max_abs": err, "out_rel_l2": rel,
+            "lse_max_abs": lerr, "outputs_checked": int(o.shape[0] * o.shape[1])}
+
+
+def main():
+    args = parse()
+    if args.layers is None:
+        args.layers = N_LAYERS if args.workload == "llama32k" else 8
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl" if args.impl == "native" else "gloo",
+                                 timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        if args.impl == "reference":
+            rc = run_reference(args, rank, world)
+        else:
+            rc = run_native(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,193 @@
+/*
+ * sa.h -- C ABI of the page-sparse decode library (sm_100a, one GPU).
+ *
+ * Query-aware top-k page-sparse decode attention over a paged KV cache, plus
+ * keep-mask prefix-cache pruning.  The sources describing the method:
+ *   [SE]  "SparseEngine" blog post (blog.ontle.kr/blog/332): hook-point paragraph
+ *         (Quest chooses, at each decode step, which pages to read from the
+ *         current query; OmniKV/DeltaKV reuse one layer's indices at later layers),
+ *         physical-vs-logical paragraph (freeing storage vs reading less), and the
+ *         Prefix-Cache Pruning paragraph (the kept part stays, the rest is freed,
+ *         the conversation-position marker is untouched).
+ *   [VX]  "Vortex" summary (gist.science/ja/paper/2606.06453), section 1: KV in
+ *         non-contiguous paged boxes; a map hands back "the top pages" without the
+ *         caller knowing where they live.
+ *   [SC]  SCBench notes (notes.yuuk.io), Tri-shape section: A-shape = attention-sink
+ *         tokens + local window; method table: Quest loads part of the KV per step.
+ *   [SSA] SubQ/SSA article (news.neo-ai.one/ja/article/2719), SSA section: exact
+ *         attention over the chosen positions; FlashAttention paragraph: no
+ *         materialised score matrix.
+ * The pages never print the formulas.  This library computes the plain method:
+ * channel-wise min/max key summaries per page; page score
+ * S(b,h,p) = max_{g in group(h)} sum_c max(q_gc*kmax_c, q_gc*kmin_c) in fp32; the
+ * budget/P best pages with sink and window pages forced in (ties -> lower page
+ * index); exact softmax attention over the selected tokens with split-KV online
+ * softmax merged by log-sum-exp.
+ *
+ * Conventions for every call:
+ *  - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or synchronises (except sa_workspace_status, which
+ *    says so).  bf16 tensors are passed as `const void*` (16-bit bf16 elements).
+ *  - Every tensor must be 16-byte aligned and densely packed in the layout given.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    enqueued asynchronously on it; calls are capturable in a CUDA graph.
+ *  - Argument errors are detected on the host before anything is launched and
+ *    returned as a negative sa_status.  Errors only the device can see (an index
+ *    out of range, a bounded wait that expired, too few free pages) are OR-ed into
+ *    the workspace status word and read with sa_workspace_status().
+ *  - Layouts (row-major, last index fastest):
+ *      q           [B][Hq][Dk]            bf16
+ *      k_cache     [n_pool][Hkv][P][Dk]   bf16   (each (page, head) block contiguous)
+ *      v_cache     [n_pool][Hkv][P][Dv]   bf16   (ignored when v_aliases_k: V is then
+ *                                                 the first Dv channels of each K row)
+ *      summ        [n_pool][Hkv][2][Dk]   bf16   row 0 = min, row 1 = max, indexed by
+ *                                                 PHYSICAL page
+ *      page_table  [B][max_pages]         int32  logical page -> physical page
+ *      seq_lens    [B]                    int32  valid tokens; logical page lp holds
+ *                                                 tokens [lp*P, lp*P+P)
+ *      sel         [B][Hkv][budget/P]     int32  ascending logical pages, -1 padded
+ *      sel_count   [B][Hkv]               int32
+ *      out         [B][Hq][Dv]            fp32   lse [B][Hq] fp32 (natural log)
+ *  - Supported geometries: grouped-query (v_aliases_k = 0): Dk = Dv in {64, 128},
+ *    G = Hq/Hkv in 1..8, Hkv <= 32; latent (v_aliases_k = 1): Hkv = 1, Dk = 576,
+ *    Dv = 512, Hq = 128.  P in {16, 32, 64}.  budget, sink, window are token counts,
+ *    multiples of P, with sink + window <= budget.  Preconditions not checked on the
+ *    device: no NaN/Inf in valid K, V, q; page_table entries of valid pages lie in
+ *    [0, n_pool).
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = -1,   /* bad pointer, size, alignment or budget/sink/window */
+  SA_ERR_UNSUPPORTED = -2,   /* geometry outside the supported set */
+  SA_ERR_WORKSPACE = -3,     /* workspace missing or smaller than the *_workspace_size */
+  SA_ERR_CUDA = -4,          /* a CUDA runtime call or a launch failed */
+  SA_ERR_DEVICE_CHECK = -5,  /* device saw an out-of-range index (status word only) */
+  SA_ERR_TIMEOUT = -6,       /* a bounded device wait expired (status word only) */
+  SA_ERR_NO_SPACE = -7       /* prune: fewer free pages than kept pages (status word) */
+} sa_status;
+
+/* Problem geometry.  n_pool = number of physical pages in k_cache/v_cache/summ. */
+typedef struct {
+  int32_t B, Hq, Hkv, Dk, Dv, P, max_pages, n_pool, v_aliases_k;
+} sa_geom;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sa_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int sa_version(void);
+
+/* ---------------------------------------------------------------------------------
+ * Workspace.  One buffer per stream (calls on one stream may share it; calls that
+ * may run concurrently need their own).  It must be zeroed once before first use
+ * (sa_workspace_init); afterwards the library keeps it consistent.  Its first 256
+ * bytes hold the status word.
+ * ------------------------------------------------------------------------------ */
+
+/* Bytes needed by sa_select_pages / sa_sparse_decode / sa_attend_selected for this
+ * geometry and budget (0 on invalid arguments). */
+size_t sa_decode_workspace_size(const sa_geom* g, int budget);
+
+/* Bytes needed by sa_prune_compact (0 on invalid arguments). */
+size_t sa_prune_workspace_size(const sa_geom* g);
+
+/* Zero `ws_bytes` bytes of workspace on `stream` (cudaMemsetAsync). */
+int sa_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the workspace status word (SA_OK or the first
+ * device-detected error) and clears it.  The only call that blocks the host. */
+int sa_workspace_status(void* ws, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (1) Per-page key summaries  [SE hook-point paragraph; VX section 1].
+ * For every valid logical page lp < ceil(seq_lens[b]/P) of every sequence, every KV
+ * head h and channel c: summ[page_table[b][lp]][h][0][c] = min over the page's
+ * valid tokens (t < seq_lens[b]) of K[t][h][c], row 1 = max.  Signed zeros order
+ * -0 < +0.  Pages referenced by no sequence are not written.  Bit-exact.
+ * ------------------------------------------------------------------------------ */
+int sa_page_summaries(const sa_geom* g, const void* k_cache, const int32_t* page_table,
+                      const int32_t* seq_lens, void* summ, void* stream);
+
+/* Same as sa_page_summaries restricted to the last `n_tail_pages` valid pages of
+ * each sequence: the decode-time update after new tokens were appended (one new
+ * token per step -> n_tail_pages = 1).  n_tail_pages >= 1. */
+int sa_update_summaries(const sa_geom* g, const void* k_cache, const int32_t* page_table,
+                        const int32_t* seq_lens, int n_tail_pages, void* summ, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (2)+(3) Page scoring and top-k selection  [SE hook-point paragraph (Quest);
+ * VX section 1 ("top pages"); SC Tri-shape section (sink + local window)].
+ * K = budget/P pages per (sequence, KV head).  If n_b = ceil(seq_lens[b]/P) <= K
+ * all n_b pages are selected.  Otherwise pages [0, sink/P) and [n_b - window/P, n_b)
+ * are forced in and the K - sink/P - window/P highest-scoring other pages join them
+ * (equal fp32 scores -> lower page index).  sel gets the ascending page list, -1
+ * after sel_count entries.  `scores` (nullable, [B][Hkv][max_pages] fp32) receives
+ * S for p < n_b and -inf beyond.  Selection is deterministic.
+ * ------------------------------------------------------------------------------ */
+int sa_select_pages(const sa_geom* g, const void* q, const void* summ,
+                    const int32_t* page_table, const int32_t* seq_lens, int budget, int sink,
+                    int window, int32_t* sel, int32_t* sel_count, float* scores, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (4) Sparse decode: selection as above, then exact attention over the tokens of
+ * the selected pages gathered through the page table  [VX section 1; SSA section;
+ * FlashAttention paragraph]:
+ *   x_t = scale * q . k_t over valid tokens t of the selected pages of KV head
+ *   hq / G;  out[b][hq] = sum_t softmax(x)_t v_t;  lse[b][hq] = log sum_t exp(x_t).
+ * A sequence with seq_len 0 gives out = 0, lse = -inf.  bf16 inputs, fp32
+ * accumulation.  sel_out / sel_count_out (nullable) receive the selection.
+ * ------------------------------------------------------------------------------ */
+int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache, const void* v_cache,
+                     const void* summ, const int32_t* page_table, const int32_t* seq_lens,
+                     int budget, int sink, int window, float scale, float* out, float* lse,
+                     int32_t* sel_out, int32_t* sel_count_out, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Attention over a given selection (sel [B][Hkv][sel_stride], ascending logical
+ * pages, sel_count [B][Hkv] <= sel_stride): the reuse of one layer's selected
+ * indices at later layers [SE hook-point paragraph, OmniKV/DeltaKV].  `budget` for
+ * the workspace size is sel_stride * P. */
+int sa_attend_selected(const sa_geom* g, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* page_table, const int32_t* seq_lens, const int32_t* sel,
+                       const int32_t* sel_count, int sel_stride, float scale, float* out,
+                       float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (5) Prefix-cache pruning  [SE physical-vs-logical and Prefix-Cache Pruning
+ * paragraphs]: physical removal of the tokens keep[b][t] == 0.
+ * For each session b in order, the kept valid tokens (t < seq_lens[b], increasing t)
+ * are numbered i = 0.. L'_b - 1 and kept token i (K and V rows of every KV head) is
+ * copied to page free_pages[off_b + i/P], slot i % P, with off_b = sum over b' < b
+ * of ceil(L'_b'/P).  Outputs: new_page_table[b][j] = free_pages[off_b + j] for
+ * j < ceil(L'_b/P), else -1; new_seq_lens[b] = L'_b; logical_len[b] = seq_lens[b]
+ * (the position marker is kept); pos_map[b][i] = original position of kept token
+ * i, -1 for i >= L'_b; summ of every new page; padding slots of a partial last page
+ * are zero.  Old pages are read, never written: the caller returns them to its
+ * allocator.  keep [B][max_pages*P] uint8, pos_map [B][max_pages*P] int32.
+ * k_dst/v_dst may be k_cache/v_cache; free pages must not be referenced by
+ * page_table.  If n_free < sum_b ceil(L'_b/P) nothing is written and the status
+ * word reports SA_ERR_NO_SPACE.  Bit-exact.
+ * ------------------------------------------------------------------------------ */
+int sa_prune_compact(const sa_geom* g, const void* k_cache, const void* v_cache,
+                     const int32_t* page_table, const int32_t* seq_lens, const uint8_t* keep,
+                     const int32_t* free_pages, int64_t n_free, void* k_dst, void* v_dst,
+                     void* summ, int32_t* new_page_table, int32_t* new_seq_lens,
+                     int32_t* pos_map, int32_t* logical_len, void* ws, size_t ws_bytes,
+                     void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */

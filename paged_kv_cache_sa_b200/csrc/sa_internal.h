@@ -1,0 +1,54 @@
+// sa_internal.h -- host-side launchers shared by the C-ABI layer (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sa.h"
+
+namespace sa {
+
+// ---- workspace carving for the decode calls ------------------------------------------
+struct DecodePlan {
+  int K;            // pages per (sequence, KV head) = budget / P
+  int G;            // query heads per KV head
+  int pps;          // selected pages handled by one attention CTA
+  int nsplit;       // attention CTAs per (sequence, KV head)
+  size_t off_scores, off_sel, off_cnt, off_part, total;
+};
+
+bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan);
+
+// ---- launchers (return the CUDA error of the launch) ----------------------------------
+cudaError_t launch_summaries(const sa_geom& g, const void* k_cache, const int32_t* page_table,
+                             const int32_t* seq_lens, void* summ, int n_tail,
+                             cudaStream_t stream);
+
+cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
+                         const int32_t* page_table, const int32_t* seq_lens, float* scores,
+                         int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_topk(const sa_geom& g, const float* scores, const int32_t* seq_lens, int K,
+                        int sink_pages, int window_pages, int32_t* sel, int32_t* sel_count,
+                        cudaStream_t stream);
+
+cudaError_t launch_attend(const sa_geom& g, const DecodePlan& plan, const void* q,
+                          const void* k_cache, const void* v_cache, const int32_t* page_table,
+                          const int32_t* seq_lens, const int32_t* sel, const int32_t* sel_count,
+                          int sel_stride, float scale, float* part, float* out, float* lse,
+                          int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_prune(const sa_geom& g, const void* k_cache, const void* v_cache,
+                         const int32_t* page_table, const int32_t* seq_lens, const uint8_t* keep,
+                         const int32_t* free_pages, int64_t n_free, void* k_dst, void* v_dst,
+                         void* summ, int32_t* new_page_table, int32_t* new_seq_lens,
+                         int32_t* pos_map, int32_t* logical_len, void* ws, cudaStream_t stream);
+
+size_t prune_workspace_bytes(const sa_geom& g);
+
+// TMA descriptor encoder from the driver (resolved once through the runtime).
+bool encode_rows_tmap(void* tmap_out, const void* base, uint64_t inner_elems, uint64_t rows,
+                      uint32_t box_inner, uint32_t box_rows);
+
+}  // namespace sa

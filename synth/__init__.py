@@ -32,7 +32,7 @@ Workloads (sizes as named by the method's target configurations):
                   (geometric lengths, mean 256) covering 20% of the middle,
                   then decode with budget 1024 (sink 64, window 512).
 
-Every workload can be shrunk (``scale_down``) for tests that must finish fast.
+Every workload can be shrunk through keyword overrides for tests that must finish fast.
 """
 
 from __future__ import annotations
@@ -58,10 +58,14 @@ POISON_BITS = {
 
 
 def f32_to_bf16(x: np.ndarray) -> np.ndarray:
-    """float32 -> bf16 bits, round to nearest even (inputs are finite)."""
+    """float32 -> bf16 bits, round to nearest even (inputs are finite, so the 32-bit
+    sum below cannot overflow: the largest finite pattern is 0xFF7FFFFF)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    u = x.view(np.uint32)
+    r = (u >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r >>= np.uint32(16)
     return r.astype(np.uint16)
 
 

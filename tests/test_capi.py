@@ -1,0 +1,65 @@
+"""The C-ABI library builds, loads without a GPU, and exports exactly what
+include/sa.h declares; the CPU-only host logic of the binding."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "sa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def libpath():
+    from paged_kv_cache_sa_b200 import build as b
+    return b.build()
+
+
+def test_header_declares_the_expected_entry_points():
+    decl = _declared()
+    for name in ("sa_page_summaries", "sa_update_summaries", "sa_select_pages",
+                 "sa_sparse_decode", "sa_attend_selected", "sa_prune_compact",
+                 "sa_decode_workspace_size", "sa_prune_workspace_size", "sa_workspace_init",
+                 "sa_workspace_status", "sa_status_string", "sa_version"):
+        assert name in decl
+
+
+def test_library_exports_every_declared_symbol(libpath):
+    lib = ctypes.CDLL(libpath)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", libpath], capture_output=True,
+                         text=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines()
+                       if ln.split() and ln.split()[-1].startswith("sa_")})
+    assert exported == _declared()
+
+
+def test_binding_loads_and_sizes_workspaces(libpath):
+    import paged_kv_cache_sa_b200 as sa
+    for name in sa.EXPORTS:
+        assert hasattr(sa.lib, name)
+    assert sa.lib.sa_version() >= 10000
+    assert sa.lib.sa_status_string(-7) == b"not enough free pages"
+    g = sa.Geometry(B=8, Hq=32, Hkv=8, Dk=128, Dv=128, P=16, max_pages=2048, n_pool=16384)
+    n = sa.decode_workspace_size(g, 2048)
+    # header + scores + selection + counts + split partials
+    assert n >= 256 + 8 * 8 * 2048 * 4 + 8 * 8 * 128 * 4
+    assert sa.decode_workspace_size(g, 2004) == 0            # budget not a multiple of P
+    bad = sa.Geometry(B=8, Hq=32, Hkv=8, Dk=96, Dv=96, P=16, max_pages=2048, n_pool=16384)
+    assert sa.decode_workspace_size(bad, 2048) == 0          # unsupported head dim
+    assert sa.prune_workspace_size(g) > 256
+
+
+def test_no_cpu_fallback_in_binding():
+    src = open(os.path.join(ROOT, "paged_kv_cache_sa_b200", "__init__.py")).read()
+    assert "import oracle" not in src and "from oracle" not in src
+    assert "numpy" not in src

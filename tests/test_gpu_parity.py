@@ -1,0 +1,254 @@
+"""GPU parity of every C-ABI entry point against the CPU oracle (needs a B200)."""
+
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import DevCase, check_attention, full_parity, run_decode, to_dev, u16
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import paged_kv_cache_sa_b200 as sa  # noqa: E402
+
+
+# ------------------------------------------------------------------------------------
+# summaries (bit-exact)
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wl,P,Dk,lens", [
+    ("tiny", 16, 64, [0, 1, 15, 16, 17, 4096]),
+    ("tiny", 32, 128, [31, 32, 33, 1000]),
+    ("tiny", 64, 128, [1, 63, 64, 65, 700]),
+    ("mla", 64, None, [1, 65, 640]),
+])
+def test_summaries_bit_exact(wl, P, Dk, lens):
+    kw = dict(B=len(lens), seq_lens=lens, P=P, identity=False, extra_pool_pages=4, poison="nan")
+    if wl == "tiny":
+        kw.update(Dk=Dk, Hkv=4, Hq=8)
+    else:
+        kw.update(Hq=128, budget=640, sink=64, window=128)
+    case = synth.decode_case(wl, **kw)
+    dc = DevCase(case)
+    sa.page_summaries(dc.g, dc.k, dc.pt, dc.sl, dc.summ)
+    ref = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    assert np.array_equal(u16(dc.summ), ref)
+
+
+def test_signed_zero_summaries():
+    case = synth.decode_case("tiny", B=1, seq_lens=[40], Hkv=1, Hq=4)
+    k = case.k_cache.copy()
+    k[:, :, :, 0] = 0x8000
+    k[:, :, 1::2, 0] = 0x0000     # -0 and +0 alternate in channel 0
+    k[:, :, :, 1] = 0x0000
+    case = dataclasses.replace(case, k_cache=k)
+    dc = DevCase(case)
+    sa.page_summaries(dc.g, dc.k, dc.pt, dc.sl, dc.summ)
+    ref = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    assert np.array_equal(u16(dc.summ), ref)
+
+
+def test_update_summaries_tail_pages():
+    # the pool already holds one appended token per sequence; summaries were computed
+    # before the append, so only each sequence's last page is stale
+    case = synth.decode_case("tiny", B=3, seq_lens=[1001, 17, 4097], Hkv=2, Hq=8,
+                             poison="nan")
+    dc = DevCase(case)
+    before = to_dev(case.seq_lens - 1)
+    sa.page_summaries(dc.g, dc.k, dc.pt, before, dc.summ)
+    sa.update_summaries(dc.g, dc.k, dc.pt, dc.sl, dc.summ, n_tail_pages=1)
+    ref = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    assert np.array_equal(u16(dc.summ), ref)
+
+
+# ------------------------------------------------------------------------------------
+# scoring + selection + attention, small end-to-end cases
+# ------------------------------------------------------------------------------------
+
+SMALL = [
+    dict(wl="tiny"),
+    dict(wl="tiny", B=3, seq_lens=[4096, 700, 50], Hkv=2, Hq=8, poison="nan"),
+    dict(wl="tiny", B=2, seq_lens=[0, 1], Hkv=1, Hq=4),
+    dict(wl="tiny", B=2, seq_lens=[513, 511], Hkv=1, Hq=4, budget=512, sink=0, window=0),
+    dict(wl="tiny", B=1, seq_lens=[3000], Hkv=1, Hq=1, budget=1024, sink=16, window=1008),
+    dict(wl="tiny", B=2, seq_lens=[5000, 2049], Hkv=2, Hq=16, P=32, budget=1024, sink=32,
+         window=256, poison="inf"),
+    dict(wl="tiny", B=2, seq_lens=[9000, 3333], Hkv=1, Hq=6, P=64, budget=1024, sink=64,
+         window=256, poison="big"),
+    dict(wl="llama32k", B=2, L=(8192, 8192), seed=12, poison="nan"),
+    dict(wl="llama32k", B=2, L=(4096, 4096), seed=13, P=32, budget=1024, sink=64, window=256),
+    dict(wl="llama32k", B=2, L=(4096, 4096), seed=14, P=64, budget=1024, sink=64, window=256),
+    dict(wl="ragged", B=2, L=(3000, 9000), seed=15, budget=1024, sink=128, window=256,
+         poison="nan"),
+]
+
+
+@pytest.mark.parametrize("kw", SMALL, ids=lambda kw: "-".join(
+    "%s%s" % (k, v if not isinstance(v, list) else len(v)) for k, v in kw.items()))
+def test_decode_parity_small(kw):
+    kw = dict(kw)
+    wl = kw.pop("wl")
+    case = synth.decode_case(wl, **kw)
+    res = run_decode(DevCase(case))
+    full_parity(case, res)
+
+
+def test_budget_covers_all_pages_equals_dense():
+    case = synth.decode_case("tiny", B=2, seq_lens=[1234, 4096], Hkv=2, Hq=8, budget=4096,
+                             poison="nan")
+    res = run_decode(DevCase(case))
+    g = case.geom
+    for b in range(g.B):
+        L = int(case.seq_lens[b])
+        for h in range(g.Hkv):
+            ks = np.concatenate([case.k_cache[case.page_table[b, p], h]
+                                 for p in range((L + 15) // 16)])[:L]
+            vs = np.concatenate([case.v_cache[case.page_table[b, p], h]
+                                 for p in range((L + 15) // 16)])[:L]
+            o, l = oracle.dense_attend(case.q[b, h * g.G:(h + 1) * g.G], ks, vs, case.scale)
+            check_attention(res["out"][b, h * g.G:(h + 1) * g.G], res["lse"][b, h * g.G:(h + 1) * g.G],
+                            o, l)
+
+
+def test_empty_sequence_outputs():
+    case = synth.decode_case("tiny", B=2, seq_lens=[0, 300], Hkv=1, Hq=4)
+    res = run_decode(DevCase(case))
+    assert (res["out"][0] == 0).all() and np.isneginf(res["lse"][0]).all()
+    assert res["cnt"][0, 0] == 0 and (res["sel"][0, 0] == -1).all()
+    full_parity(case, res)
+
+
+def test_attend_selected_reuses_indices():
+    # one layer's selection reused at another layer (different q, K, V; same lengths)
+    c1 = synth.decode_case("llama32k", B=2, L=(4096, 4096), seed=31)
+    c2 = synth.decode_case("llama32k", B=2, L=(4096, 4096), seed=32)
+    d1, d2 = DevCase(c1), DevCase(c2)
+    r1 = run_decode(d1, scores=False)
+    ws = sa.Workspace.for_decode(d2.g, c2.budget)
+    sel = to_dev(r1["sel"])
+    cnt = to_dev(r1["cnt"])
+    out, lse = sa.attend_selected(d2.g, d2.q, d2.k, d2.v, d2.pt, d2.sl, sel, cnt, c2.scale, ws)
+    assert ws.status() == sa.SA_OK
+    ro, rl = oracle.attend(c2.geom, c2.q, c2.k_cache, c2.v_cache, c2.page_table, c2.seq_lens,
+                           r1["sel"], r1["cnt"], c2.scale)
+    check_attention(out.cpu().numpy(), lse.cpu().numpy(), ro, rl)
+
+
+def test_deterministic_bitwise():
+    case = synth.decode_case("llama32k", B=2, L=(8192, 8192), seed=17)
+    dc = DevCase(case)
+    a = run_decode(dc)
+    b = run_decode(dc)
+    for k in ("summ", "sel", "cnt", "out", "lse", "scores"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+# ------------------------------------------------------------------------------------
+# invalid arguments are rejected on the host before any launch
+# ------------------------------------------------------------------------------------
+
+def test_invalid_arguments():
+    case = synth.decode_case("tiny")
+    dc = DevCase(case)
+    g = dc.g
+    ws = sa.Workspace.for_decode(g, case.budget)
+    with pytest.raises(sa.SaError) as e:
+        sa.sparse_decode(g, dc.q, dc.k, dc.v, dc.summ, dc.pt, dc.sl, case.budget, 512, 64,
+                         case.scale, ws)
+    assert e.value.status == -1                        # sink + window > budget
+    with pytest.raises(sa.SaError) as e:
+        sa.sparse_decode(g, dc.q, dc.k, dc.v, dc.summ, dc.pt, dc.sl, 500, 16, 64, case.scale, ws)
+    assert e.value.status == -1                        # budget not a multiple of P
+    small = sa.Workspace(256)
+    with pytest.raises(sa.SaError) as e:
+        sa.sparse_decode(g, dc.q, dc.k, dc.v, dc.summ, dc.pt, dc.sl, case.budget, 16, 64,
+                         case.scale, small)
+    assert e.value.status == -3                        # workspace too small
+    bad = dataclasses.replace(g, Dk=96, Dv=96)
+    with pytest.raises(sa.SaError) as e:
+        sa.page_summaries(bad, dc.k, dc.pt, dc.sl, dc.summ)
+    assert e.value.status == -2                        # unsupported head dim
+    bad = dataclasses.replace(g, Hq=5, Hkv=2)
+    with pytest.raises(sa.SaError) as e:
+        sa.page_summaries(bad, dc.k, dc.pt, dc.sl, dc.summ)
+    assert e.value.status == -1                        # Hq % Hkv != 0
+    assert ws.status() == sa.SA_OK
+
+
+# ------------------------------------------------------------------------------------
+# prefix-cache pruning (bit-exact)
+# ------------------------------------------------------------------------------------
+
+def _run_prune(pc, n_free=None):
+    d = pc.decode
+    g = sa.Geometry.of(d.geom)
+    k, v = to_dev(d.k_cache), to_dev(d.v_cache) if d.v_cache is not None else None
+    summ = torch.zeros((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device="cuda")
+    ws = sa.Workspace.for_prune(g)
+    fp = to_dev(pc.free_pages if n_free is None else pc.free_pages[:n_free])
+    npt, nsl, pos, ll = sa.prune_compact(g, k, v, to_dev(d.page_table), to_dev(d.seq_lens),
+                                         to_dev(pc.keep), fp, k, v, summ, ws)
+    st = ws.status()
+    return st, dict(k_dst=u16(k), v_dst=u16(v) if v is not None else None, summ=u16(summ),
+                    new_page_table=npt.cpu().numpy(), new_seq_lens=nsl.cpu().numpy(),
+                    pos_map=pos.cpu().numpy(), logical_len=ll.cpu().numpy())
+
+
+@pytest.mark.parametrize("kw", [
+    dict(B=3, seq_lens=[3000, 2200, 5000], Hkv=2, Hq=8),
+    dict(B=4, seq_lens=[0, 1, 17, 9000], Hkv=8, Hq=32, extra_free=5),
+    dict(B=2, seq_lens=[4100, 300], Hkv=8, Hq=32, P=32),
+    dict(B=2, seq_lens=[8200, 100], Hkv=4, Hq=8, P=64),
+    dict(B=2, seq_lens=[3000, 700], Hkv=2, Hq=8, keep_all=True),
+    dict(B=2, seq_lens=[3000, 700], Hkv=2, Hq=8, keep_none=True),
+])
+def test_prune_bit_exact(kw):
+    pc = synth.prune_case("prune", **kw)
+    st, r = _run_prune(pc)
+    assert st == sa.SA_OK
+    d = pc.decode
+    ref = oracle.prune_compact(d.geom, d.k_cache, d.v_cache, d.page_table, d.seq_lens, pc.keep,
+                               pc.free_pages)
+    summ_ref = ref["summ"]
+    for key in ("new_page_table", "new_seq_lens", "pos_map", "logical_len", "k_dst", "v_dst"):
+        assert np.array_equal(r[key], ref[key]), key
+    # the oracle writes summaries of new pages only; so does the library
+    assert np.array_equal(r["summ"], summ_ref)
+
+
+def test_prune_latent_pool():
+    pc = synth.prune_case("mla", B=2, seq_lens=[3000, 640], Hq=128, budget=640, sink=64,
+                          window=128)
+    st, r = _run_prune(pc)
+    assert st == sa.SA_OK
+    d = pc.decode
+    ref = oracle.prune_compact(d.geom, d.k_cache, None, d.page_table, d.seq_lens, pc.keep,
+                               pc.free_pages)
+    for key in ("new_page_table", "new_seq_lens", "pos_map", "logical_len", "k_dst", "summ"):
+        assert np.array_equal(r[key], ref[key]), key
+
+
+def test_prune_reports_no_space_and_writes_nothing():
+    pc = synth.prune_case("prune", B=2, seq_lens=[3000, 2200], Hkv=2, Hq=8)
+    d = pc.decode
+    st, r = _run_prune(pc, n_free=len(pc.free_pages) - 1)
+    assert st == -7                                    # SA_ERR_NO_SPACE
+    assert np.array_equal(r["k_dst"], d.k_cache)       # pool untouched
+    assert (r["summ"] == 0).all()
+
+
+def test_decode_after_prune():
+    pc = synth.prune_case("prune", B=3, seq_lens=[9000, 12000, 5000], Hkv=8, Hq=32)
+    st, r = _run_prune(pc)
+    assert st == sa.SA_OK
+    d = pc.decode
+    comp = dataclasses.replace(d, k_cache=r["k_dst"], v_cache=r["v_dst"],
+                               page_table=r["new_page_table"], seq_lens=r["new_seq_lens"])
+    res = run_decode(DevCase(comp))
+    full_parity(comp, res)
