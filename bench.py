@@ -2,11 +2,11 @@
 
 One step = one decode step of a 32-layer model with Llama-3.1-8B attention geometry
 (batch 8, 32 query / 8 KV heads, head dim 128, 32768 tokens per sequence, page 16,
-token budget 2048 = sink 64 + window 512 + top-k): for every layer, the summary of
-each sequence's newest page is refreshed (sa_update_summaries), every page is scored
-and the top pages selected (sa_select_pages: scoring + top-k kernels), and attention
-runs over the gathered pages (sa_attend_selected: split-KV attention + merge) -- the
-two halves of sa_sparse_decode, called separately so the bench can time each.
+token budget 2048 = sink 64 + window 512 + top-k): for every layer, sa_select_pages
+refreshes the summary of each sequence's newest page, scores every page and selects
+the top pages (one fused kernel), and sa_attend_selected runs split-KV attention over
+the gathered pages with the merge fused in (one persistent kernel) -- the two halves
+of sa_sparse_decode, called separately so the bench can time each.
 Every layer owns its own KV pool, so a step touches ~4.3 GB (> L2) and nothing is
 served from L2 across layers.
 
@@ -242,6 +242,7 @@ def run_native(args, rank, world, dist):
     ws = sa.Workspace.for_decode(g, case.budget)
     sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device=dev)
     cnt = torch.empty((g.B, g.Hkv), dtype=torch.int32, device=dev)
+    phys = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device=dev)
     outs = [torch.empty((g.B, g.Hq, g.Dv), dtype=torch.float32, device=dev) for _ in range(L_layers)]
     lses = [torch.empty((g.B, g.Hq), dtype=torch.float32, device=dev) for _ in range(L_layers)]
     torch.cuda.synchronize()
@@ -253,13 +254,13 @@ def run_native(args, rank, world, dist):
         for l in range(L_layers):
             if with_events:
                 ev[l][0].record()
-            sa.update_summaries(g, ks[l], pt, sl, summs[l], 1)
             sa.select_pages(g, qs[l], summs[l], pt, sl, case.budget, case.sink, case.window, ws,
-                            sel=sel, sel_count=cnt)
+                            sel=sel, sel_count=cnt, k_cache=ks[l], n_tail_refresh=1,
+                            sel_phys=phys)
             if with_events:
                 ev[l][1].record()
             sa.attend_selected(g, qs[l], ks[l], vs[l], pt, sl, sel, cnt, case.scale, ws,
-                               out=outs[l], lse=lses[l])
+                               out=outs[l], lse=lses[l], sel_phys=phys)
             if with_events:
                 ev[l][2].record()
 
@@ -365,8 +366,7 @@ def run_native(args, rank, world, dist):
     cpu_v, cpu_done, cpu_t = (None, 0, 0.0)
     if world == 1:
         cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    launches_per_layer = 4 + (1 if plan_nsplit(g, case.budget, sms) > 1 else 0)
+    launches_per_layer = 2  # score+select (with the tail refresh), attention (+merge)
     line = {
         "metric": "sparse-decode seq*heads/s",
         "value": value,
@@ -395,8 +395,7 @@ def run_native(args, rank, world, dist):
             "algorithmic_bytes_per_layer": sel_b + att_b + upd_b,
         },
         "roofline": {
-            "kernel": "attend_gqa_kernel+merge_kernel" if dom_is_att
-            else "update+score_gqa_kernel+topk_kernel",
+            "kernel": "attend_gqa_kernel" if dom_is_att else "score_select_kernel",
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "peak_kind": peak_kind + " (burst copy)",
             "traffic": None,
@@ -413,15 +412,6 @@ def run_native(args, rank, world, dist):
     }
     print(json.dumps(line, default=_json_default), flush=True)
     return 0
-
-
-def plan_nsplit(g, budget, sm_count):
-    """Attention CTAs per (sequence, KV head) as the library plans them (same rule)."""
-    K = budget // g.P
-    units = g.B * g.Hkv
-    ns = max(1, min(K, (4 * sm_count + units - 1) // units))
-    pps = min(256, (((K + ns - 1) // ns) + 3) & ~3)
-    return (K + pps - 1) // pps
 
 
 def full_size_parity(case, out0, lse0, sel, cnt, sa, g, ks, vs, qs, summs, pt, sl, ws, dev):

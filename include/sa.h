@@ -88,10 +88,14 @@ const char* sa_status_string(int status);
 int sa_version(void);
 
 /* ---------------------------------------------------------------------------------
- * Workspace.  One buffer per stream (calls on one stream may share it; calls that
- * may run concurrently need their own).  It must be zeroed once before first use
- * (sa_workspace_init); afterwards the library keeps it consistent.  Its first 256
- * bytes hold the status word.
+ * Workspace.  One buffer per (stream, geometry, budget): calls on one stream with the
+ * same geometry and budget may share it; calls that may run concurrently, or that use
+ * another geometry or budget, need their own (or a fresh sa_workspace_init in between,
+ * since the layout of its counters depends on the geometry).  It must be zeroed once
+ * before first use (sa_workspace_init); afterwards the library keeps it consistent
+ * (its arrival counters return to zero at the end of every call).  Its first 256 bytes
+ * hold the status word.  A call that reported SA_ERR_TIMEOUT may leave counters
+ * behind: zero the workspace again before reusing it.
  * ------------------------------------------------------------------------------ */
 
 /* Bytes needed by sa_select_pages / sa_sparse_decode / sa_attend_selected for this
@@ -133,11 +137,18 @@ int sa_update_summaries(const sa_geom* g, const void* k_cache, const int32_t* pa
  * (equal fp32 scores -> lower page index).  sel gets the ascending page list, -1
  * after sel_count entries.  `scores` (nullable, [B][Hkv][max_pages] fp32) receives
  * S for p < n_b and -inf beyond.  Selection is deterministic.
+ * Decode-time refresh: with n_tail_refresh in 1..16 (k_cache then required), the
+ * summaries of the last n_tail_refresh pages of every sequence are first recomputed
+ * from k_cache -- the pages that just received appended tokens -- and written to
+ * summ, exactly as sa_update_summaries would; 0 leaves summ untouched.
+ * sel_phys (nullable, [B][Hkv][budget/P] int32) receives page_table[b][sel[b][h][i]]
+ * for each selected entry (-1 after sel_count): handing it to sa_attend_selected
+ * saves that call one dependent page-table lookup.
  * ------------------------------------------------------------------------------ */
-int sa_select_pages(const sa_geom* g, const void* q, const void* summ,
-                    const int32_t* page_table, const int32_t* seq_lens, int budget, int sink,
-                    int window, int32_t* sel, int32_t* sel_count, float* scores, void* ws,
-                    size_t ws_bytes, void* stream);
+int sa_select_pages(const sa_geom* g, const void* q, void* summ, const int32_t* page_table,
+                    const int32_t* seq_lens, int budget, int sink, int window,
+                    const void* k_cache, int n_tail_refresh, int32_t* sel, int32_t* sel_count,
+                    int32_t* sel_phys, float* scores, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * (4) Sparse decode: selection as above, then exact attention over the tokens of
@@ -146,22 +157,29 @@ int sa_select_pages(const sa_geom* g, const void* q, const void* summ,
  *   x_t = scale * q . k_t over valid tokens t of the selected pages of KV head
  *   hq / G;  out[b][hq] = sum_t softmax(x)_t v_t;  lse[b][hq] = log sum_t exp(x_t).
  * A sequence with seq_len 0 gives out = 0, lse = -inf.  bf16 inputs, fp32
- * accumulation.  sel_out / sel_count_out (nullable) receive the selection.
+ * accumulation.  sel_out / sel_count_out (nullable) receive the selection;
+ * n_tail_refresh as in sa_select_pages.
  * ------------------------------------------------------------------------------ */
 int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache, const void* v_cache,
-                     const void* summ, const int32_t* page_table, const int32_t* seq_lens,
-                     int budget, int sink, int window, float scale, float* out, float* lse,
-                     int32_t* sel_out, int32_t* sel_count_out, void* ws, size_t ws_bytes,
-                     void* stream);
+                     void* summ, const int32_t* page_table, const int32_t* seq_lens, int budget,
+                     int sink, int window, int n_tail_refresh, float scale, float* out,
+                     float* lse, int32_t* sel_out, int32_t* sel_count_out, void* ws,
+                     size_t ws_bytes, void* stream);
 
 /* Attention over a given selection (sel [B][Hkv][sel_stride], ascending logical
  * pages, sel_count [B][Hkv] <= sel_stride): the reuse of one layer's selected
  * indices at later layers [SE hook-point paragraph, OmniKV/DeltaKV].  `budget` for
- * the workspace size is sel_stride * P. */
+ * the workspace size is sel_stride * P.  sel_phys (nullable) holds the physical page
+ * of each entry as written by sa_select_pages; passing it also states that the
+ * selection was made by sa_select_pages for these seq_lens with budget
+ * sel_stride * P, so that sel_count[b][h] == min(ceil(seq_lens[b] / P), sel_stride)
+ * (the kernel then derives the counts from seq_lens and starts earlier).  Without
+ * sel_phys the page table and sel_count are read. */
 int sa_attend_selected(const sa_geom* g, const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* page_table, const int32_t* seq_lens, const int32_t* sel,
-                       const int32_t* sel_count, int sel_stride, float scale, float* out,
-                       float* lse, void* ws, size_t ws_bytes, void* stream);
+                       const int32_t* sel_count, const int32_t* sel_phys, int sel_stride,
+                       float scale, float* out, float* lse, void* ws, size_t ws_bytes,
+                       void* stream);
 
 /* ---------------------------------------------------------------------------------
  * (5) Prefix-cache pruning  [SE physical-vs-logical and Prefix-Cache Pruning

@@ -75,11 +75,11 @@ class Geometry:
         return cls(g.B, g.Hq, g.Hkv, g.Dk, g.Dv, g.P, g.max_pages, g.n_pool, g.v_aliases_k)
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
         raise ImportError("libsa.so is not built (%s); run __graft_entry__.build() or "
-                          "python paged_kv_cache_sa_b200/build.py" % LIB_PATH)
-    lib = ctypes.CDLL(LIB_PATH)
+                          "python paged_kv_cache_sa_b200/build.py" % path)
+    lib = ctypes.CDLL(path)
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     G = ctypes.POINTER(sa_geom)
     sig = {
@@ -91,11 +91,12 @@ def _load() -> ctypes.CDLL:
         "sa_workspace_status": ([vp, vp], i32),
         "sa_page_summaries": ([G, vp, vp, vp, vp, vp], i32),
         "sa_update_summaries": ([G, vp, vp, vp, i32, vp, vp], i32),
-        "sa_select_pages": ([G, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp], i32),
-        "sa_sparse_decode": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.c_float, vp, vp,
-                              vp, vp, vp, sz, vp], i32),
-        "sa_attend_selected": ([G, vp, vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp, vp,
-                                sz, vp], i32),
+        "sa_select_pages": ([G, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, sz,
+                             vp], i32),
+        "sa_sparse_decode": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, vp,
+                              vp, vp, vp, vp, sz, vp], i32),
+        "sa_attend_selected": ([G, vp, vp, vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp,
+                                vp, sz, vp], i32),
         "sa_prune_compact": ([G, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                               vp], i32),
     }
@@ -180,7 +181,11 @@ def update_summaries(geom: Geometry, k_cache, page_table, seq_lens, summ, n_tail
 
 
 def select_pages(geom: Geometry, q, summ, page_table, seq_lens, budget, sink, window,
-                 ws: Workspace, sel=None, sel_count=None, scores=None, stream=None):
+                 ws: Workspace, sel=None, sel_count=None, scores=None, k_cache=None,
+                 n_tail_refresh: int = 0, sel_phys=None, stream=None):
+    """Score every page and select the top pages (plus sink and window pages).
+    With ``n_tail_refresh`` > 0 the last pages' summaries are first recomputed from
+    ``k_cache`` (the decode-time update after an append)."""
     K = budget // geom.P
     dev = q.device
     if sel is None:
@@ -189,15 +194,17 @@ def select_pages(geom: Geometry, q, summ, page_table, seq_lens, budget, sink, wi
         sel_count = torch.empty((geom.B, geom.Hkv), dtype=torch.int32, device=dev)
     g = geom.c()
     _check(lib.sa_select_pages(ctypes.byref(g), _ptr(q), _ptr(summ), _ptr(page_table),
-                               _ptr(seq_lens), int(budget), int(sink), int(window), _ptr(sel),
-                               _ptr(sel_count), _ptr(scores), _ptr(ws.buf), ws.nbytes,
-                               _stream(stream)), "sa_select_pages")
+                               _ptr(seq_lens), int(budget), int(sink), int(window),
+                               _ptr(k_cache), int(n_tail_refresh), _ptr(sel), _ptr(sel_count),
+                               _ptr(sel_phys), _ptr(scores), _ptr(ws.buf), ws.nbytes,
+                               _stream(stream)),
+           "sa_select_pages")
     return sel, sel_count
 
 
 def sparse_decode(geom: Geometry, q, k_cache, v_cache, summ, page_table, seq_lens, budget, sink,
                   window, scale, ws: Workspace, out=None, lse=None, sel_out=None,
-                  sel_count_out=None, stream=None):
+                  sel_count_out=None, n_tail_refresh: int = 0, stream=None):
     dev = q.device
     if out is None:
         out = torch.empty((geom.B, geom.Hq, geom.Dv), dtype=torch.float32, device=dev)
@@ -206,14 +213,14 @@ def sparse_decode(geom: Geometry, q, k_cache, v_cache, summ, page_table, seq_len
     g = geom.c()
     _check(lib.sa_sparse_decode(ctypes.byref(g), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(summ),
                                 _ptr(page_table), _ptr(seq_lens), int(budget), int(sink),
-                                int(window), float(scale), _ptr(out), _ptr(lse), _ptr(sel_out),
-                                _ptr(sel_count_out), _ptr(ws.buf), ws.nbytes, _stream(stream)),
-           "sa_sparse_decode")
+                                int(window), int(n_tail_refresh), float(scale), _ptr(out),
+                                _ptr(lse), _ptr(sel_out), _ptr(sel_count_out), _ptr(ws.buf),
+                                ws.nbytes, _stream(stream)), "sa_sparse_decode")
     return out, lse
 
 
 def attend_selected(geom: Geometry, q, k_cache, v_cache, page_table, seq_lens, sel, sel_count,
-                    scale, ws: Workspace, out=None, lse=None, stream=None):
+                    scale, ws: Workspace, out=None, lse=None, sel_phys=None, stream=None):
     dev = q.device
     if out is None:
         out = torch.empty((geom.B, geom.Hq, geom.Dv), dtype=torch.float32, device=dev)
@@ -222,7 +229,8 @@ def attend_selected(geom: Geometry, q, k_cache, v_cache, page_table, seq_lens, s
     g = geom.c()
     _check(lib.sa_attend_selected(ctypes.byref(g), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                   _ptr(page_table), _ptr(seq_lens), _ptr(sel), _ptr(sel_count),
-                                  int(sel.shape[-1]), float(scale), _ptr(out), _ptr(lse),
+                                  _ptr(sel_phys), int(sel.shape[-1]), float(scale), _ptr(out),
+                                  _ptr(lse),
                                   _ptr(ws.buf), ws.nbytes, _stream(stream)), "sa_attend_selected")
     return out, lse
 

@@ -27,7 +27,7 @@ static int sm_count() {
 
 static bool is_gqa(const sa_geom& g) {
   return !g.v_aliases_k && (g.Dk == 64 || g.Dk == 128) && g.Dv == g.Dk && g.Hq % g.Hkv == 0 &&
-         g.Hq / g.Hkv >= 1 && g.Hq / g.Hkv <= 8 && g.Hkv <= 32;
+         g.Hq / g.Hkv >= 1 && g.Hq / g.Hkv <= 8 && g.Hkv <= 32 && attend_supported(g);
 }
 
 static bool is_latent(const sa_geom& g) {
@@ -59,16 +59,7 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   DecodePlan p{};
   p.K = budget / g.P;
   p.G = g.Hq / g.Hkv;
-  const int units = g.B * g.Hkv;
-  const int target = 4 * sm_count();
-  int ns = (target + units - 1) / units;
-  if (ns < 1) ns = 1;
-  if (ns > p.K) ns = p.K;
-  int pps = (p.K + ns - 1) / ns;
-  pps = (pps + 3) & ~3;  // whole rounds of the four consumer warps
-  if (pps > 256) pps = 256;
-  p.pps = pps;
-  p.nsplit = (p.K + pps - 1) / pps;
+  p.n_cta = attend_ctas(g, p.K, sm_count());
   size_t off = 256;  // status header
   p.off_scores = off;
   off += up256((size_t)g.B * g.Hkv * g.max_pages * 4);
@@ -76,8 +67,14 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   off += up256((size_t)g.B * g.Hkv * p.K * 4);
   p.off_cnt = off;
   off += up256((size_t)g.B * g.Hkv * 4);
+  p.off_phys = off;
+  off += up256((size_t)g.B * g.Hkv * p.K * 4);
+  p.off_arrive = off;
+  off += up256((size_t)g.B * g.Hkv * 4);
+  p.off_merge = off;
+  off += up256((size_t)g.B * g.Hkv * 4);
   p.off_part = off;
-  if (p.nsplit > 1) off += up256((size_t)g.B * g.Hkv * p.nsplit * p.G * (g.Dv + 2) * 4);
+  off += up256(attend_partial_floats(g, p.n_cta) * 4);
   p.total = off;
   *plan = p;
   return true;
@@ -192,42 +189,76 @@ SA_EXPORT int sa_update_summaries(const sa_geom* g, const void* k_cache, const i
 }
 
 // scoring + selection into (sel, cnt); shared by select and decode
-static int run_select(const sa_geom& g, const DecodePlan& plan, const void* q, const void* summ,
-                      const int32_t* page_table, const int32_t* seq_lens, int sink, int window,
-                      int32_t* sel, int32_t* cnt, float* scores, int32_t* status,
-                      cudaStream_t s) {
+static int run_select(const sa_geom& g, const DecodePlan& plan, uint8_t* w, const void* q,
+                      void* summ, const void* k_cache, int n_tail, const int32_t* page_table,
+                      const int32_t* seq_lens, int sink, int window, int32_t* sel, int32_t* cnt,
+                      int32_t* phys, float* scores, cudaStream_t s) {
   if (!is_gqa(g)) return SA_ERR_UNSUPPORTED;
-  cudaError_t e = launch_score(g, q, summ, page_table, seq_lens, scores, status, s);
-  if (e != cudaSuccess) return SA_ERR_CUDA;
-  e = launch_topk(g, scores, seq_lens, plan.K, sink / g.P, window / g.P, sel, cnt, s);
-  return cuda_status(e);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
+  return cuda_status(launch_score_select(
+      g, q, summ, n_tail > 0 ? k_cache : nullptr, n_tail, page_table, seq_lens, scores,
+      reinterpret_cast<uint32_t*>(w + plan.off_arrive), plan.K, sink / g.P, window / g.P, sel,
+      cnt, phys, &hdr->status_bits, s));
 }
 
-SA_EXPORT int sa_select_pages(const sa_geom* g, const void* q, const void* summ,
+static int run_attend(const sa_geom& g, const DecodePlan& plan, uint8_t* w, const void* q,
+                      const void* k_cache, const void* v_cache, const int32_t* page_table,
+                      const int32_t* seq_lens, const int32_t* sel, const int32_t* cnt,
+                      const int32_t* sel_phys, int sel_stride, float scale, float* out,
+                      float* lse, cudaStream_t s) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
+  AttendCall c;
+  c.q = q;
+  c.k_cache = k_cache;
+  c.v_cache = v_cache;
+  c.page_table = page_table;
+  c.seq_lens = seq_lens;
+  c.sel = sel;
+  c.sel_count = cnt;
+  c.sel_phys = sel_phys;
+  c.sel_stride = sel_stride;
+  c.scale = scale;
+  c.part = reinterpret_cast<float*>(w + plan.off_part);
+  c.merge_cnt = reinterpret_cast<uint32_t*>(w + plan.off_merge);
+  c.out = out;
+  c.lse = lse;
+  c.status = &hdr->status_bits;
+  c.n_cta = plan.n_cta;
+  c.counts_from_lens = sel_phys != nullptr;
+  return cuda_status(launch_attend(g, c, s));
+}
+
+SA_EXPORT int sa_select_pages(const sa_geom* g, const void* q, void* summ,
                               const int32_t* page_table, const int32_t* seq_lens, int budget,
-                              int sink, int window, int32_t* sel, int32_t* sel_count,
+                              int sink, int window, const void* k_cache, int n_tail_refresh,
+                              int32_t* sel, int32_t* sel_count, int32_t* sel_phys,
                               float* scores, void* ws, size_t ws_bytes, void* stream) {
   int st = check_geom(g);
   if (st != SA_OK) return st;
   if ((st = check_budget(*g, budget, sink, window)) != SA_OK) return st;
   if (!q || !summ || !page_table || !seq_lens || !sel || !sel_count) return SA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(summ)) return SA_ERR_INVALID_ARG;
+  if (n_tail_refresh < 0 || n_tail_refresh > 16 || (n_tail_refresh > 0 && !k_cache))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(summ) || (k_cache && !aligned16(k_cache)))
+    return SA_ERR_INVALID_ARG;
   if ((size_t)g->max_pages * 4 > 200 * 1024) return SA_ERR_UNSUPPORTED;
+  if (!is_gqa(*g)) return SA_ERR_UNSUPPORTED;
   DecodePlan plan;
   make_decode_plan(*g, budget, &plan);
   if (!ws || ws_bytes < plan.total || !aligned16(ws)) return SA_ERR_WORKSPACE;
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* sc = scores ? scores : reinterpret_cast<float*>(w + plan.off_scores);
-  return run_select(*g, plan, q, summ, page_table, seq_lens, sink, window, sel, sel_count, sc,
-                    &reinterpret_cast<WsHeader*>(w)->status_bits,
-                    static_cast<cudaStream_t>(stream));
+  int32_t* ph = sel_phys ? sel_phys : reinterpret_cast<int32_t*>(w + plan.off_phys);
+  return run_select(*g, plan, w, q, summ, k_cache, n_tail_refresh, page_table, seq_lens, sink,
+                    window, sel, sel_count, ph, sc, static_cast<cudaStream_t>(stream));
 }
 
 SA_EXPORT int sa_attend_selected(const sa_geom* g, const void* q, const void* k_cache,
                                  const void* v_cache, const int32_t* page_table,
                                  const int32_t* seq_lens, const int32_t* sel,
-                                 const int32_t* sel_count, int sel_stride, float scale,
-                                 float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+                                 const int32_t* sel_count, const int32_t* sel_phys,
+                                 int sel_stride, float scale, float* out, float* lse, void* ws,
+                                 size_t ws_bytes, void* stream) {
   int st = check_geom(g);
   if (st != SA_OK) return st;
   if (!is_gqa(*g)) return SA_ERR_UNSUPPORTED;
@@ -240,24 +271,23 @@ SA_EXPORT int sa_attend_selected(const sa_geom* g, const void* q, const void* k_
   DecodePlan plan;
   make_decode_plan(*g, sel_stride * g->P, &plan);
   if (!ws || ws_bytes < plan.total || !aligned16(ws)) return SA_ERR_WORKSPACE;
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
-  return cuda_status(launch_attend(*g, plan, q, k_cache, vc, page_table, seq_lens, sel, sel_count,
-                                   sel_stride, scale, reinterpret_cast<float*>(w + plan.off_part),
-                                   out, lse, &hdr->status_bits,
-                                   static_cast<cudaStream_t>(stream)));
+  return run_attend(*g, plan, static_cast<uint8_t*>(ws), q, k_cache, vc, page_table, seq_lens,
+                    sel, sel_count, sel_phys, sel_stride, scale, out, lse,
+                    static_cast<cudaStream_t>(stream));
 }
 
 SA_EXPORT int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache,
-                               const void* v_cache, const void* summ, const int32_t* page_table,
+                               const void* v_cache, void* summ, const int32_t* page_table,
                                const int32_t* seq_lens, int budget, int sink, int window,
-                               float scale, float* out, float* lse, int32_t* sel_out,
-                               int32_t* sel_count_out, void* ws, size_t ws_bytes, void* stream) {
+                               int n_tail_refresh, float scale, float* out, float* lse,
+                               int32_t* sel_out, int32_t* sel_count_out, void* ws,
+                               size_t ws_bytes, void* stream) {
   int st = check_geom(g);
   if (st != SA_OK) return st;
   if ((st = check_budget(*g, budget, sink, window)) != SA_OK) return st;
   if (!q || !k_cache || !summ || !page_table || !seq_lens || !out || !lse)
     return SA_ERR_INVALID_ARG;
+  if (n_tail_refresh < 0 || n_tail_refresh > 16) return SA_ERR_INVALID_ARG;
   if (!g->v_aliases_k && !v_cache) return SA_ERR_INVALID_ARG;
   const void* vc = g->v_aliases_k ? k_cache : v_cache;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(vc) || !aligned16(summ))
@@ -268,18 +298,16 @@ SA_EXPORT int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_ca
   make_decode_plan(*g, budget, &plan);
   if (!ws || ws_bytes < plan.total || !aligned16(ws)) return SA_ERR_WORKSPACE;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
   int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + plan.off_sel);
   int32_t* cnt = sel_count_out ? sel_count_out : reinterpret_cast<int32_t*>(w + plan.off_cnt);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = run_select(*g, plan, q, summ, page_table, seq_lens, sink, window, sel, cnt,
-                  reinterpret_cast<float*>(w + plan.off_scores), &hdr->status_bits, s);
+  st = run_select(*g, plan, w, q, summ, k_cache, n_tail_refresh, page_table, seq_lens, sink,
+                  window, sel, cnt, reinterpret_cast<int32_t*>(w + plan.off_phys),
+                  reinterpret_cast<float*>(w + plan.off_scores), s);
   if (st != SA_OK) return st;
-  return cuda_status(launch_attend(*g, plan, q, k_cache, vc, page_table, seq_lens, sel, cnt,
-                                   plan.K, scale, reinterpret_cast<float*>(w + plan.off_part), out,
-                                   lse, &hdr->status_bits, s));
+  return run_attend(*g, plan, w, q, k_cache, vc, page_table, seq_lens, sel, cnt,
+                    reinterpret_cast<int32_t*>(w + plan.off_phys), plan.K, scale, out, lse, s);
 }
-
 SA_EXPORT int sa_prune_compact(const sa_geom* g, const void* k_cache, const void* v_cache,
                                const int32_t* page_table, const int32_t* seq_lens,
                                const uint8_t* keep, const int32_t* free_pages, int64_t n_free,

@@ -11,11 +11,10 @@ namespace sa {
 
 // ---- workspace carving for the decode calls ------------------------------------------
 struct DecodePlan {
-  int K;            // pages per (sequence, KV head) = budget / P
-  int G;            // query heads per KV head
-  int pps;          // selected pages handled by one attention CTA
-  int nsplit;       // attention CTAs per (sequence, KV head)
-  size_t off_scores, off_sel, off_cnt, off_part, total;
+  int K;      // pages per (sequence, KV head) = budget / P
+  int G;      // query heads per KV head
+  int n_cta;  // attention CTAs (one per SM, more for very large selections)
+  size_t off_scores, off_sel, off_cnt, off_phys, off_arrive, off_merge, off_part, total;
 };
 
 bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan);
@@ -25,19 +24,37 @@ cudaError_t launch_summaries(const sa_geom& g, const void* k_cache, const int32_
                              const int32_t* seq_lens, void* summ, int n_tail,
                              cudaStream_t stream);
 
-cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
-                         const int32_t* page_table, const int32_t* seq_lens, float* scores,
-                         int32_t* status, cudaStream_t stream);
+cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
+                                int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+                                float* scores, uint32_t* arrivals, int K, int sink_pages,
+                                int window_pages, int32_t* sel, int32_t* sel_count,
+                                int32_t* sel_phys, int32_t* status, cudaStream_t stream);
 
-cudaError_t launch_topk(const sa_geom& g, const float* scores, const int32_t* seq_lens, int K,
-                        int sink_pages, int window_pages, int32_t* sel, int32_t* sel_count,
-                        cudaStream_t stream);
+struct AttendCall {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const int32_t* sel;
+  const int32_t* sel_count;
+  const int32_t* sel_phys;  // physical pages of sel (nullable: looked up in page_table)
+  int sel_stride;
+  float scale;
+  float* part;
+  uint32_t* merge_cnt;
+  float* out;
+  float* lse;
+  int32_t* status;
+  int n_cta;
+  int counts_from_lens;  // the selection came from this library for these seq_lens
+};
 
-cudaError_t launch_attend(const sa_geom& g, const DecodePlan& plan, const void* q,
-                          const void* k_cache, const void* v_cache, const int32_t* page_table,
-                          const int32_t* seq_lens, const int32_t* sel, const int32_t* sel_count,
-                          int sel_stride, float scale, float* part, float* out, float* lse,
-                          int32_t* status, cudaStream_t stream);
+int attend_ctas(const sa_geom& g, int K, int sms);
+size_t attend_partial_floats(const sa_geom& g, int n_cta);
+bool attend_supported(const sa_geom& g);
+
+cudaError_t launch_attend(const sa_geom& g, const AttendCall& c, cudaStream_t stream);
 
 cudaError_t launch_prune(const sa_geom& g, const void* k_cache, const void* v_cache,
                          const int32_t* page_table, const int32_t* seq_lens, const uint8_t* keep,

@@ -67,6 +67,40 @@ def test_update_summaries_tail_pages():
     assert np.array_equal(u16(dc.summ), ref)
 
 
+def test_fused_tail_refresh_in_selection():
+    # stale summaries for the newest page; select_pages refreshes them from K first
+    case = synth.decode_case("llama32k", B=3, seq_lens=[4097, 3000, 2064], seed=41,
+                             poison="nan")
+    dc = DevCase(case)
+    before = to_dev(np.maximum(case.seq_lens - 1, 0))
+    sa.page_summaries(dc.g, dc.k, dc.pt, before, dc.summ)
+    ws = sa.Workspace.for_decode(dc.g, case.budget)
+    sel, cnt = sa.select_pages(dc.g, dc.q, dc.summ, dc.pt, dc.sl, case.budget, case.sink,
+                               case.window, ws, k_cache=dc.k, n_tail_refresh=1)
+    assert ws.status() == sa.SA_OK
+    ref = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    assert np.array_equal(u16(dc.summ), ref)
+    sc = oracle.page_scores(case.geom, case.q, ref, case.page_table, case.seq_lens)
+    osel, ocnt = oracle.select_pages(case.geom, sc, case.seq_lens, case.budget, case.sink,
+                                     case.window)
+    from parity import check_selection
+    check_selection(case.geom, case.seq_lens, case.budget, case.sink, case.window, sc, osel,
+                    ocnt, sel.cpu().numpy(), cnt.cpu().numpy())
+
+
+def test_workspace_reuse_across_calls():
+    # counters inside a workspace return to zero after every call: many calls in a row
+    # on the same workspace (and interleaved with another geometry's workspace) stay exact
+    c1 = synth.decode_case("llama32k", B=2, L=(4096, 4096), seed=51)
+    c2 = synth.decode_case("llama32k", B=2, seq_lens=[1000, 4000], seed=52)
+    d1, d2 = DevCase(c1), DevCase(c2)
+    w1 = sa.Workspace.for_decode(d1.g, c1.budget)
+    w2 = sa.Workspace.for_decode(d2.g, c2.budget)
+    for _ in range(3):
+        full_parity(c1, run_decode(d1, ws=w1))
+        full_parity(c2, run_decode(d2, ws=w2))
+
+
 # ------------------------------------------------------------------------------------
 # scoring + selection + attention, small end-to-end cases
 # ------------------------------------------------------------------------------------
