@@ -35,6 +35,7 @@ namespace sa {
 constexpr int kMaxUnitsPerCta = 256;  // slice table capacity
 constexpr int kMaxPairs = 4096;       // pairs (sequence x KV head) per call
 constexpr int kSmemLimit = 227 * 1024;
+constexpr int kGmax = 8;  // query heads per KV head
 
 // NC consumer warps, SPW stages (units in flight) per consumer warp
 template <int D, int P, int NC, int SPW>
@@ -106,52 +107,65 @@ __device__ __forceinline__ int find_pair(const int* pre, int n_pairs, int u) {
   return lo;
 }
 
-// Merge n states (each [G][HS]: O row, m, l) at buf into one.  dst == nullptr: write the
-// normalised result to out ([G][D]) and lse ([G]); otherwise store the merged state at dst
-// (global or shared; dst may be buf itself, state 0).  One warp; compact loops.
+// Merge n (<= 32) states (each [G][HS]: O row, m, l) at buf into one.  dst == nullptr:
+// write the normalised result to out ([G][D]) and lse ([G]); otherwise store the merged
+// state at dst (global or shared; dst may be buf itself, state 0).  One warp.  All
+// heads are reduced into registers first and written after a single __syncwarp: a
+// __syncwarp between global stores would wait for them to complete.
 template <int D>
 __device__ __noinline__ void merge_states(float* buf, int n, int STATE, int G, int lane,
                                           float* dst, float* out, float* lse) {
   constexpr int HS = D + 4;
+  float acc[kGmax][D / 32], mst[kGmax], lsm[kGmax];
+#pragma unroll
+  for (int gi = 0; gi < kGmax; ++gi) {
+    mst[gi] = -INFINITY;
+    lsm[gi] = 0.f;
+#pragma unroll
+    for (int q4 = 0; q4 < D / 32; ++q4) acc[gi][q4] = 0.f;
+    if (gi < G) {
+      // lane w < n holds state w's (m, l); its weight is 2^(m_w - m*)
+      const float mw = lane < n ? buf[lane * STATE + gi * HS + D] : -INFINITY;
+      const float lw = lane < n ? buf[lane * STATE + gi * HS + D + 1] : 0.f;
+      float mstar = mw;
+#pragma unroll
+      for (int off = 16; off; off >>= 1)
+        mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, off));
+      const float fw = (mw == -INFINITY) ? 0.f : fast_exp2(mw - mstar);
+      float lsum = lw * fw;
+#pragma unroll
+      for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+      mst[gi] = mstar;
+      lsm[gi] = lsum;
 #pragma unroll 1
-  for (int gi = 0; gi < G; ++gi) {
-    // lane w < n holds state w's (m, l); its weight 2^(m_w - m*)
-    const float mw = lane < n ? buf[lane * STATE + gi * HS + D] : -INFINITY;
-    const float lw = lane < n ? buf[lane * STATE + gi * HS + D + 1] : 0.f;
-    float mstar = mw;
+      for (int w = 0; w < n; ++w) {
+        const float f = __shfl_sync(0xffffffffu, fw, w);
+        const float* row = buf + w * STATE + gi * HS;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, off));
-    const float fw = (mw == -INFINITY) ? 0.f : fast_exp2(mw - mstar);
-    float lsum = lw * fw;
-#pragma unroll
-    for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    float acc[D / 32];
-#pragma unroll
-    for (int q4 = 0; q4 < D / 32; ++q4) acc[q4] = 0.f;
-#pragma unroll 1
-    for (int w = 0; w < n; ++w) {
-      const float f = __shfl_sync(0xffffffffu, fw, w);
-      const float* row = buf + w * STATE + gi * HS;
-#pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) acc[q4] += row[lane + 32 * q4] * f;
+        for (int q4 = 0; q4 < D / 32; ++q4) acc[gi][q4] += row[lane + 32 * q4] * f;
+      }
     }
-    __syncwarp();
+  }
+  __syncwarp();  // every read of buf is done before dst (possibly buf) is written
+#pragma unroll
+  for (int gi = 0; gi < kGmax; ++gi) {
+    if (gi >= G) continue;
     if (dst) {
       float* drow = dst + gi * HS;
 #pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) drow[lane + 32 * q4] = acc[q4];
+      for (int q4 = 0; q4 < D / 32; ++q4) drow[lane + 32 * q4] = acc[gi][q4];
       if (lane == 0) {
-        drow[D] = mstar;
-        drow[D + 1] = lsum;
+        drow[D] = mst[gi];
+        drow[D + 1] = lsm[gi];
       }
     } else {
+      const float lsum = lsm[gi];
       float* o = out + gi * D;
 #pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) o[lane + 32 * q4] = lsum > 0.f ? acc[q4] / lsum : 0.f;
+      for (int q4 = 0; q4 < D / 32; ++q4) o[lane + 32 * q4] = lsum > 0.f ? acc[gi][q4] / lsum : 0.f;
       if (lane == 0)
-        lse[gi] = lsum > 0.f ? (mstar + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+        lse[gi] = lsum > 0.f ? (mst[gi] + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
     }
-    __syncwarp();
   }
 }
 
