@@ -1,46 +1,51 @@
-// sa_attend.cu -- gathered split-KV attention over the selected pages, merge fused in.
+// sa_attend.cu -- gathered split-KV attention over the selected pages, then the merge.
 //
 // Method: exact softmax attention over the tokens of the selected pages (SubQ/SSA
 // article, SSA section: exact attention on the chosen positions), reached through the
 // page table without the caller knowing where pages live (Vortex summary, section 1),
 // with an online softmax that never materialises the score row (FlashAttention
-// paragraph of the same article); the pages are split across CTAs and the partial
-// results merged by log-sum-exp.
+// paragraph of the same article); the pages are split across warps and the partial
+// results merged by log-sum-exp (flash-decoding style split-KV).
 //
 // Work layout.  The selected pages of all (sequence, KV head) pairs, cut into units of
-// 16 tokens, form one flattened list (pair-major, ascending page order).  CTA c (one
-// per SM) takes the contiguous slice [c*W, (c+1)*W) of it, W = ceil(total / #CTAs), so
-// every SM streams the same number of bytes whatever the sequence lengths.
-//  * Producer warp: builds the slice's tables in shared memory (pair prefix sums, then
-//    per unit: pair, physical page, valid tokens -- all lanes' loads in flight together)
-//    and splits the slice into per-pair segments.  Then lane w feeds consumer warp w's
-//    private ring of stages with units w, w+8, w+16, ...: 2-D TMA tile loads of the
-//    unit's K and V (128-byte swizzle, mbarrier transaction counts, no multicast).
-//  * 8 consumer warps, per unit: S = Q K^T on m16n8k16 tensor-core tiles (the G <= 8
+// 16 tokens, form one flattened list (pair-major, ascending page order).  Warp w of CTA c
+// (global warp gw = c * NC + w) takes the contiguous range [gw*W, (gw+1)*W) of it,
+// W = ceil(total / #warps), so every SM streams the same number of bytes whatever the
+// sequence lengths.
+//  * Producer warp: builds the CTA's tables in shared memory (pair prefix sums, then per
+//    unit: pair, first K/V row, valid tokens -- all lanes' loads in flight together).
+//    Then lane w feeds consumer warp w's private ring of stages with its units in order:
+//    2-D TMA tile loads of the unit's K and V (128-byte swizzle, mbarrier transaction
+//    counts, no multicast).
+//  * NC consumer warps, per unit: S = Q K^T on m16n8k16 tensor-core tiles (the G <= 8
 //    query heads are the M side; K fragments come from the swizzled stage with
 //    conflict-free 16-byte shared loads in a permuted channel order that Q's fragments
 //    share), online softmax in registers (base 2, scale folded in), then O^T += V^T P^T
 //    with the channels as the M side (V^T fragments by ldmatrix.trans, the S
-//    accumulators are directly the P^T operand).
-//  * At the end of every segment the 8 warps' (m, l, O) meet in shared memory; one warp
-//    merges them.  A pair covered by one CTA is written out directly; otherwise the
-//    CTA's partial goes to the workspace and the last CTA of the pair (atomic counter,
-//    no waiting) merges the 2-4 partials in CTA order (deterministic).
+//    accumulators are directly the P^T operand).  When the pair changes, or the range
+//    ends, a pair lying wholly inside the warp's range is normalised and written out;
+//    a pair cut by the range boundary leaves its (m, l, O) state in the workspace
+//    (slot 0: the pair began before the range, slot 1: it goes on after it).
+//  * attend_merge_kernel (launched programmatically dependent, so its CTAs are resident
+//    before the attention grid ends) merges the states of every cut pair in range order
+//    (deterministic), and writes the empty pairs (out = 0, lse = -inf).
+// No global memory traffic but the K/V stream happens while a warp streams: a load or
+// fence issued behind the SM's deep queue of TMA reads waits for that whole queue.
 // HBM-bound: bytes per selected token and KV head = (Dk + Dv) * 2.
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
 namespace sa {
 
-constexpr int kMaxUnitsPerCta = 256;  // slice table capacity
+constexpr int kMaxUnitsPerCta = 256;  // CTA table capacity
 constexpr int kMaxPairs = 4096;       // pairs (sequence x KV head) per call
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kGmax = 8;  // query heads per KV head
+constexpr int kAttnWarps = 8;  // consumer warps per CTA
 
 // NC consumer warps, SPW stages (units in flight) per consumer warp
 template <int D, int P, int NC, int SPW>
 struct AttnShape {
-  static constexpr int THREADS = (NC + 2) * 32;  // consumers, producer, merger
+  static constexpr int THREADS = (NC + 1) * 32;  // consumers, producer
   static constexpr int CT = 16;                         // tokens per unit
   static constexpr int UPP = P / CT;                    // units per page
   static constexpr int HALVES = D / 64;                 // 128-B halves per row
@@ -50,12 +55,11 @@ struct AttnShape {
   static constexpr int NST = SPW * NC;
   static constexpr int MT = D / 16;  // PV m-tiles (channels)
   static constexpr int JQ = D / 32;  // 16-byte Q/K chunks per lane
-  static constexpr int HS = D + 4;  // floats per query head in a state: O[D], m, l, pad
-  // dynamic shared memory: stages | combine states [2][NC][G][HS] | pair prefix | unit and
-  // segment tables
-  static size_t smem_bytes(int G, int n_pairs) {
-    return 1024 + (size_t)NST * STAGE_BYTES + (size_t)2 * NC * G * HS * 4 +
-           (size_t)(n_pairs + 1) * 4 + (size_t)7 * kMaxUnitsPerCta * 4 + 16;
+  static constexpr int HS = D + 4;   // floats per query head in a state: O[D], m, l, pad
+  // dynamic shared memory: stages | pair prefix | unit tables
+  static size_t smem_bytes(int n_pairs) {
+    return 1024 + (size_t)NST * STAGE_BYTES + (size_t)(n_pairs + 1) * 4 +
+           (size_t)3 * kMaxUnitsPerCta * 4 + 16;
   }
 };
 
@@ -66,8 +70,8 @@ struct AttnArgs {
   const int32_t* sel;
   const int32_t* sel_count;
   const int32_t* sel_phys;  // physical page of each selected entry (nullable)
-  float* part;              // [#CTAs][2][G][D+2] CTA partials
-  uint32_t* merge_cnt;      // [B*Hkv] arrivals of CTA partials (zero between calls)
+  float* part;              // [#warps][2][G][D+4] states of cut pairs
+  int32_t* pre_out;         // [n_pairs + 1] pair prefix of units (written by CTA 0)
   float* out;
   float* lse;
   int32_t* status;
@@ -90,10 +94,6 @@ __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-__device__ __forceinline__ void named_arrive(int id, int n) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // the pair owning flattened unit u: largest p with pre[p] <= u
 __device__ __forceinline__ int find_pair(const int* pre, int n_pairs, int u) {
   int lo = 0, hi = n_pairs - 1;
@@ -107,94 +107,30 @@ __device__ __forceinline__ int find_pair(const int* pre, int n_pairs, int u) {
   return lo;
 }
 
-// Merge n (<= 32) states (each [G][HS]: O row, m, l) at buf into one.  dst == nullptr:
-// write the normalised result to out ([G][D]) and lse ([G]); otherwise store the merged
-// state at dst (global or shared; dst may be buf itself, state 0).  One warp.  All
-// heads are reduced into registers first and written after a single __syncwarp: a
-// __syncwarp between global stores would wait for them to complete.
-template <int D>
-__device__ __noinline__ void merge_states(float* buf, int n, int STATE, int G, int lane,
-                                          float* dst, float* out, float* lse) {
-  constexpr int HS = D + 4;
-  float acc[kGmax][D / 32], mst[kGmax], lsm[kGmax];
-#pragma unroll
-  for (int gi = 0; gi < kGmax; ++gi) {
-    mst[gi] = -INFINITY;
-    lsm[gi] = 0.f;
-#pragma unroll
-    for (int q4 = 0; q4 < D / 32; ++q4) acc[gi][q4] = 0.f;
-    if (gi < G) {
-      // lane w < n holds state w's (m, l); its weight is 2^(m_w - m*)
-      const float mw = lane < n ? buf[lane * STATE + gi * HS + D] : -INFINITY;
-      const float lw = lane < n ? buf[lane * STATE + gi * HS + D + 1] : 0.f;
-      float mstar = mw;
-#pragma unroll
-      for (int off = 16; off; off >>= 1)
-        mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, off));
-      const float fw = (mw == -INFINITY) ? 0.f : fast_exp2(mw - mstar);
-      float lsum = lw * fw;
-#pragma unroll
-      for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-      mst[gi] = mstar;
-      lsm[gi] = lsum;
-#pragma unroll 1
-      for (int w = 0; w < n; ++w) {
-        const float f = __shfl_sync(0xffffffffu, fw, w);
-        const float* row = buf + w * STATE + gi * HS;
-#pragma unroll
-        for (int q4 = 0; q4 < D / 32; ++q4) acc[gi][q4] += row[lane + 32 * q4] * f;
-      }
-    }
-  }
-  __syncwarp();  // every read of buf is done before dst (possibly buf) is written
-#pragma unroll
-  for (int gi = 0; gi < kGmax; ++gi) {
-    if (gi >= G) continue;
-    if (dst) {
-      float* drow = dst + gi * HS;
-#pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) drow[lane + 32 * q4] = acc[gi][q4];
-      if (lane == 0) {
-        drow[D] = mst[gi];
-        drow[D + 1] = lsm[gi];
-      }
-    } else {
-      const float lsum = lsm[gi];
-      float* o = out + gi * D;
-#pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) o[lane + 32 * q4] = lsum > 0.f ? acc[gi][q4] / lsum : 0.f;
-      if (lane == 0)
-        lse[gi] = lsum > 0.f ? (mst[gi] + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
-    }
-  }
+// Units per warp for `total` units over `n_warps` warps (at least 1).
+__device__ __forceinline__ int units_per_warp(int total, int n_warps) {
+  return max(1, (total + n_warps - 1) / n_warps);
 }
 
 template <int D, int P, int NC, int SPW>
-__global__ void __launch_bounds__((NC + 2) * 32, 1)
+__global__ void __launch_bounds__((NC + 1) * 32, 1)
     attend_gqa_kernel(const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
   using S = AttnShape<D, P, NC, SPW>;
-  constexpr int kConsumers = NC;
-  constexpr int kAttnThreads = S::THREADS;
+  constexpr int kThreads = S::THREADS;
+  constexpr int HS = S::HS;
   const int G = a.Hq / a.Hkv;
   const int n_pairs = a.B * a.Hkv;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int HS = S::HS;
-  const int STATE = G * HS;  // floats of one warp's state
-  float* comb = reinterpret_cast<float*>(stages + S::NST * S::STAGE_BYTES);
-  int* pre = reinterpret_cast<int*>(comb + 2 * NC * STATE);  // [n_pairs + 1]
-  int* u_phys = pre + n_pairs + 1;                        // physical page, -1 = masked
-  int* u_row = u_phys + kMaxUnitsPerCta;                  // first K/V row in the pool
-  int* u_nv = u_row + kMaxUnitsPerCta;                    // valid tokens of the unit
-  int* u_pair = u_nv + kMaxUnitsPerCta;
-  int* seg_start = u_pair + kMaxUnitsPerCta;              // [kMaxUnitsPerCta + 1]
-  int* seg_pair = seg_start + kMaxUnitsPerCta + 1;
-  int* seg_ord = seg_pair + kMaxUnitsPerCta;             // processing order of segments
+  int* pre = reinterpret_cast<int*>(stages + S::NST * S::STAGE_BYTES);  // [n_pairs + 1]
+  int* u_row = pre + n_pairs + 1;        // first K/V row of the unit in the pool
+  int* u_nv = u_row + kMaxUnitsPerCta;   // valid tokens of the unit (0: skip)
+  int* u_pair = u_nv + kMaxUnitsPerCta;  // pair of the unit
   __shared__ __align__(8) uint64_t full_bar[S::NST];
   __shared__ __align__(8) uint64_t empty_bar[S::NST];
-  __shared__ int sh_n_seg, sh_U0, sh_W, abort_flag;
+  __shared__ int sh_nu, sh_U0, sh_W, abort_flag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, n_cta = gridDim.x;
@@ -209,7 +145,7 @@ __global__ void __launch_bounds__((NC + 2) * 32, 1)
   }
   __syncthreads();
 
-  if (warp == kConsumers) {
+  if (warp == NC) {
     // ===================== producer warp: tables =====================
     // 1. pair prefix sums of units.  A selection made by this library holds exactly
     //    min(ceil(seq_len / P), K) pages per pair, known from the sequence lengths alone,
@@ -240,11 +176,11 @@ __global__ void __launch_bounds__((NC + 2) * 32, 1)
     }
     if (lane == 0) pre[n_pairs] = carry;
     const int total = carry;
-    const int W = max(1, (total + n_cta - 1) / n_cta);
-    const int U0 = min(total, c * W);
-    const int nu = min(total, U0 + W) - U0;
+    const int W = units_per_warp(total, n_cta * NC);
+    const int U0 = min(total, c * NC * W);
+    const int nu = min(total, U0 + NC * W) - U0;
     __syncwarp();
-    // 2. per unit of the slice: its pair and place in the pair's selection
+    // 2. per unit of the CTA's range: its pair and place in the pair's selection
     constexpr int R = kMaxUnitsPerCta / 32;
     int up[R], ui[R], upart[R], lp[R], ph[R], L[R];
 #pragma unroll
@@ -262,34 +198,12 @@ __global__ void __launch_bounds__((NC + 2) * 32, 1)
         u_pair[j] = p;
       }
     }
-    __syncwarp();
-    // 3. segments: maximal runs of one pair
-    int n_seg = 0;
-    for (int j0 = 0; j0 < nu; j0 += 32) {
-      const int j = j0 + lane;
-      const bool start = j < nu && (j == 0 || u_pair[j] != u_pair[j - 1]);
-      const unsigned m = __ballot_sync(0xffffffffu, start);
-      if (start) {
-        const int k = n_seg + __popc(m & ((1u << lane) - 1));
-        seg_start[k] = j;
-        seg_pair[k] = u_pair[j];
-      }
-      n_seg += __popc(m);
-    }
-    // 4. the selection itself comes from the previous kernel of the stream
+    // 3. the selection itself comes from the previous kernel of the stream
     if (a.counts_from_lens) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
-    // pairs with nothing selected (seq_len 0): out = 0, lse = -inf
-    for (int p = c * 32 + lane; p < n_pairs; p += n_cta * 32) {
-      if (pre[p + 1] != pre[p]) continue;
-      const int b = p / a.Hkv, h = p % a.Hkv;
-      for (int gi = 0; gi < G; ++gi) {
-        float* o = a.out + ((size_t)b * a.Hq + h * G + gi) * D;
-        for (int ch = 0; ch < D; ++ch) o[ch] = 0.f;
-        a.lse[(size_t)b * a.Hq + h * G + gi] = -INFINITY;
-      }
-    }
-    // 5. physical page and valid tokens of every unit (all loads in flight together)
+    if (c == 0)
+      for (int p = lane; p <= n_pairs; p += 32) a.pre_out[p] = pre[p];
+    // 4. first K/V row and valid tokens of every unit (all loads in flight together)
 #pragma unroll
     for (int k = 0; k < R; ++k) {
       const int j = lane + 32 * k;
@@ -316,53 +230,35 @@ __global__ void __launch_bounds__((NC + 2) * 32, 1)
         } else {
           nv = max(0, min(S::CT, Lb - lp[k] * P - upart[k] * S::CT));
         }
-        u_phys[j] = phys;
         u_row[j] = phys >= 0 ? (phys * a.Hkv + h) * P + upart[k] * S::CT : 0;
         u_nv[j] = nv;
       }
     }
     if (lane == 0) {
-      seg_start[n_seg] = nu;
-      sh_n_seg = n_seg;
+      sh_nu = nu;
       sh_U0 = U0;
       sh_W = W;
     }
-    // processing order: the slice's first and last segments (the ones shared with the
-    // neighbouring CTAs) come first, so the cross-CTA merges finish while the whole
-    // pairs in between are still streaming
-    for (int i = lane; i < n_seg; i += 32)
-      seg_ord[i] = i == 0 ? 0 : (i == 1 ? n_seg - 1 : i - 1);
     __syncwarp();
-    named_bar(1, kAttnThreads);  // tables ready
+    named_bar(1, kThreads);  // tables ready
 
     // ===================== producer warp: TMA issue =====================
     if (lane == 0) {
       prefetch_tmap(&kmap);
       prefetch_tmap(&vmap);
     }
+    // lane w < NC feeds consumer warp w: units [w*W, min(nu, (w+1)*W)) in order
+    int j = lane * W;
+    const int j_end = lane < NC ? min(nu, j + W) : 0;
     int k = 0;  // units issued to consumer warp `lane`
-    // next unit of consumer warp `lane` in processing order: units j == lane (mod NC)
-    // of segment seg_ord[oi]
-    int oi = 0, j = -1;
-    auto advance = [&]() {
-      while (oi < n_seg) {
-        const int sg = seg_ord[oi];
-        const int sa_ = seg_start[sg], sb_ = seg_start[sg + 1];
-        j = j < 0 ? sa_ + ((lane - sa_) % kConsumers + kConsumers) % kConsumers : j + kConsumers;
-        if (j < sb_) return;
-        ++oi;
-        j = -1;
-      }
-    };
-    if (lane < kConsumers) advance();
     uint64_t t_idle = 0;
     for (;;) {
-      const bool busy = lane < kConsumers && oi < n_seg;
+      const bool busy = j < j_end;
       bool issued = false;
       if (busy) {
-        const int st = lane + kConsumers * (k % SPW);
+        const int st = lane + NC * (k % SPW);
         if (k < SPW || mbar_test(&empty_bar[st], ((k / SPW) - 1) & 1)) {
-          if (u_phys[j] >= 0 && u_nv[j] > 0) {
+          if (u_nv[j] > 0) {
             uint8_t* kdst = stages + st * S::STAGE_BYTES;
             uint8_t* vdst = kdst + S::KV_BYTES;
             const int row = u_row[j];
@@ -376,7 +272,7 @@ __global__ void __launch_bounds__((NC + 2) * 32, 1)
             mbar_arrive(&full_bar[st]);
           }
           ++k;
-          advance();
+          ++j;
           issued = true;
         }
       }
@@ -396,221 +292,176 @@ __global__ void __launch_bounds__((NC + 2) * 32, 1)
         }
       }
     }
-  } else if (warp < kConsumers) {
+  } else {
     // ===================== consumer warps =====================
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    named_bar(1, kAttnThreads);  // tables ready
+    named_bar(1, kThreads);  // tables ready
     const int r = lane >> 2, t = lane & 3;
     const uint32_t stage0 = smem_u32(stages);
-    const int n_seg = sh_n_seg;
+    const int W = sh_W, U0 = sh_U0, nu = sh_nu;
+    const int j0 = min(nu, warp * W), j1 = min(nu, j0 + W);
+    const int gw = c * NC + warp;          // global warp: owner of states part[gw][0..1]
+    const int wa = U0 + j0, wb = U0 + j1;  // the warp's range in the flattened list
     // ldmatrix.x4.trans row of this lane: tokens 0-7 (lanes 0-15) or 8-15 (16-31),
     // channel chunk 2*i2 (lanes 0-7, 16-23) or 2*i2 + 1 (8-15, 24-31)
     const int vtok = (lane & 7) + ((lane >> 4) << 3);
     const int vsub = (lane >> 3) & 1;
-    int kc = 0;  // units consumed by this warp
     uint4 qa[S::JQ];
-    for (int sgi = 0; sgi < n_seg; ++sgi) {
-      const int sg = seg_ord[sgi];  // segment processed in this round
-      const int p = seg_pair[sg];
-      const int sa_ = seg_start[sg], sb_ = seg_start[sg + 1];
-      const int b = p / a.Hkv, h = p % a.Hkv;
-      if (r < G) {
-        const uint4* qrow =
-            reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + h * G + r) * D);
-#pragma unroll
-        for (int j = 0; j < S::JQ; ++j) qa[j] = qrow[qk_chunk(j, t)];
-      } else {
-#pragma unroll
-        for (int j = 0; j < S::JQ; ++j) qa[j] = make_uint4(0, 0, 0, 0);
-      }
-      float m_run = -INFINITY, l_run = 0.f;
-      float o[S::MT][4];
-#pragma unroll
-      for (int i = 0; i < S::MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-      // my units of this segment: j = warp + 8i within [sa_, sb_)
-      const int first = sa_ + ((warp - sa_) % kConsumers + kConsumers) % kConsumers;
-      for (int j = first; j < sb_; j += kConsumers, ++kc) {
-        const int st = warp + kConsumers * (kc % SPW);
-        bool ok = !*(volatile int*)&abort_flag;
-        if (ok && !mbar_wait(&full_bar[st], (kc / SPW) & 1)) {
-          report(a.status, SA_ERR_TIMEOUT);
-          atomicExch(&abort_flag, 1);
-          ok = false;
-        }
-        const int nv = ok ? u_nv[j] : 0;
-        const uint32_t kbase = stage0 + st * S::STAGE_BYTES;
-        const uint32_t vbase = kbase + S::KV_BYTES;
-        if (nv > 0 && nv < S::CT) {
-          // rows past the valid tokens may hold anything: zero them in V (p = 0 there)
-          uint8_t* vrow = stages + st * S::STAGE_BYTES + S::KV_BYTES;
-          for (int e = lane; e < (S::CT - nv) * S::HALVES * 8; e += 32) {
-            const int row = nv + e / (S::HALVES * 8), cc = e % (S::HALVES * 8);
-            *reinterpret_cast<uint4*>(vrow + (cc >> 3) * S::HALF_BYTES + row * 128 +
-                                      ((cc & 7) << 4)) = make_uint4(0, 0, 0, 0);
-          }
-          // the next TMA copy into this stage must not overtake these plain stores
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-        }
-        if (nv > 0) {
-          // ---- S = Q K^T for 16 tokens (two n-tiles of 8) ----
-          float sc[2][4];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-            const int row = nt * 8 + r;
-#pragma unroll
-            for (int jj = 0; jj < S::JQ; ++jj) {
-              const int lc = qk_chunk(jj, t);
-              const uint32_t addr =
-                  kbase + (lc >> 3) * S::HALF_BYTES + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
-              const uint4 kv = lds_v4(addr);
-              mma_bf16_16816(sc[nt], qa[jj].x, 0u, qa[jj].y, 0u, kv.x, kv.y);
-              mma_bf16_16816(sc[nt], qa[jj].z, 0u, qa[jj].w, 0u, kv.z, kv.w);
-            }
-          }
-          // ---- online softmax: row = query head r; lane t: tokens 2t,2t+1,8+2t,9+2t ----
-          float x[4];
-          x[0] = 2 * t < nv ? sc[0][0] * a.scale_log2 : -INFINITY;
-          x[1] = 2 * t + 1 < nv ? sc[0][1] * a.scale_log2 : -INFINITY;
-          x[2] = 2 * t + 8 < nv ? sc[1][0] * a.scale_log2 : -INFINITY;
-          x[3] = 2 * t + 9 < nv ? sc[1][1] * a.scale_log2 : -INFINITY;
-          float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-          const float m_new = fmaxf(m_run, mt);  // finite: token 0 of a unit is valid
-          const float alpha = fast_exp2(m_run - m_new);
-          float pr[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - m_new);
-          l_run = l_run * alpha + (pr[0] + pr[1]) + (pr[2] + pr[3]);
-          m_run = m_new;
-          const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * t) * 4);
-          const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) * 4);
-          const uint32_t pb0 = pack_bf16(pr[0], pr[1]);
-          const uint32_t pb1 = pack_bf16(pr[2], pr[3]);
-          // ---- O^T += V^T P^T: m-tile i2 = channels 16 i2 .. 16 i2 + 15 ----
-#pragma unroll
-          for (int i2 = 0; i2 < S::MT; ++i2) {
-            o[i2][0] *= al0;
-            o[i2][1] *= al1;
-            o[i2][2] *= al0;
-            o[i2][3] *= al1;
-            const int lc = 2 * i2 + vsub;
-            const uint32_t addr = vbase + (lc >> 3) * S::HALF_BYTES + vtok * 128 +
-                                  (((lc & 7) ^ (vtok & 7)) << 4);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_trans(addr, a0, a1, a2, a3);
-            mma_bf16_16816(o[i2], a0, a1, a2, a3, pb0, pb1);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[st]);
-      }
-      // ---- segment end: hand this warp's state to the merger (buffer sgi & 1) ----
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[S::MT][4];
+    int cur = -1;  // pair of the running state
+
+    // Write the running state of pair `p`: normalised output when the pair lies wholly
+    // inside the warp's range, else the raw (m, l, O) state for the merge kernel.
+    auto finish = [&](int p) {
       float lt = l_run;
       lt += __shfl_xor_sync(0xffffffffu, lt, 1);
       lt += __shfl_xor_sync(0xffffffffu, lt, 2);
-      // buffer sgi & 1 was last used for segment sgi - 2: wait until it is merged
-      if (sgi >= 2) named_bar(4 + (sgi & 1), (kConsumers + 1) * 32);
-      float* my = comb + ((size_t)(sgi & 1) * kConsumers + warp) * STATE;
-      // per warp: [G][HS] = O row, m, l
-#pragma unroll
-      for (int i2 = 0; i2 < S::MT; ++i2) {
-        const int c0 = 16 * i2 + r, c1 = 16 * i2 + 8 + r;
-        if (2 * t < G) {
-          my[(2 * t) * HS + c0] = o[i2][0];
-          my[(2 * t) * HS + c1] = o[i2][2];
-        }
-        if (2 * t + 1 < G) {
-          my[(2 * t + 1) * HS + c0] = o[i2][1];
-          my[(2 * t + 1) * HS + c1] = o[i2][3];
-        }
-      }
-      if (t == 0 && r < G) {
-        my[r * HS + D] = m_run;
-        my[r * HS + D + 1] = lt;
-      }
-      __threadfence_block();
-      named_arrive(2 + (sgi & 1), (kConsumers + 1) * 32);
-    }
-  } else {
-    // ===================== merger warp =====================
-    named_bar(1, kAttnThreads);  // tables ready
-    const int n_seg = sh_n_seg, U0 = sh_U0, W = sh_W;
-    for (int sgi = 0; sgi < n_seg; ++sgi) {
-      const int sg = seg_ord[sgi];
-      const int p = seg_pair[sg];
-      const int sa_ = seg_start[sg], sb_ = seg_start[sg + 1];
+      const int ua = pre[p], ub = pre[p + 1];
       const int b = p / a.Hkv, h = p % a.Hkv;
-      named_bar(2 + (sgi & 1), (kConsumers + 1) * 32);  // the NC states are written
-      float* comb_s = comb + (size_t)(sgi & 1) * kConsumers * STATE;
-      do {
-      // ---- merge the NC states of this segment (compact code: it runs once per
-      //      segment, so it is kept small rather than unrolled) ----
-      const int ua = U0 + sa_, ub = U0 + sb_;
-      const bool whole = ua == pre[p] && ub == pre[p + 1];
-      const int slot = sg == 0 ? 0 : 1;  // only a slice's first / last segment is partial
-      float* dst = whole ? nullptr : a.part + ((size_t)c * 2 + slot) * STATE;
-      merge_states<D>(comb_s, kConsumers, STATE, G, lane, dst,
-                      a.out + ((size_t)b * a.Hq + h * G) * D, a.lse + (size_t)b * a.Hq + h * G);
-      if (whole) break;
-      // ---- a pair shared with other CTAs: the last CTA to arrive merges ----
-      __threadfence();
-      __syncwarp();
-      const int c_first = pre[p] / W, c_last = (pre[p + 1] - 1) / W;
-      uint32_t old = 0;
-      if (lane == 0) old = atomicAdd(a.merge_cnt + p, 1u);
-      old = __shfl_sync(0xffffffffu, old, 0);
-      if (old != (uint32_t)(c_last - c_first)) break;
-      __threadfence();
-      // Fold the pair's CTA partials, up to NC at a time, into the combine area (now idle)
-      // and merge them there in CTA order (deterministic).  The running result of the
-      // previous chunks is carried as one more state.
-      {
-        const int np = c_last - c_first + 1;
-        const int vec = STATE / 4;  // 16-byte vectors per state
-        int carried = 0;            // states already in the buffer (the running result)
-        for (int i0 = 0; i0 < np;) {
-          const int n = min(kConsumers - carried, np - i0);
-          __syncwarp();
-          // eight loads in flight per lane before any of them is stored
-#pragma unroll 1
-          for (int e0 = lane; e0 < n * vec; e0 += 8 * 32) {
-            float4 v[8];
+      if (ua >= wa && ub <= wb) {
+        // heads 2t and 2t+1 of this lane's O^T fragments: their l lives in the lanes
+        // with r == head
+        const float l0 = __shfl_sync(0xffffffffu, lt, (2 * t) * 4);
+        const float l1 = __shfl_sync(0xffffffffu, lt, (2 * t + 1) * 4);
+        const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
+        const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+        float* ob = a.out + ((size_t)b * a.Hq + h * G) * D;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int e = e0 + 32 * u;
-              if (e < n * vec) {
-                const int cc = c_first + i0 + e / vec;
-                const int sl = cc * W < pre[p] ? 1 : 0;
-                v[u] = __ldcg(reinterpret_cast<const float4*>(
-                                  a.part + ((size_t)cc * 2 + sl) * STATE) + e % vec);
-              }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int e = e0 + 32 * u;
-              if (e < n * vec)
-                reinterpret_cast<float4*>(comb_s + (size_t)(carried + e / vec) * STATE)[e % vec] =
-                    v[u];
-            }
+        for (int i2 = 0; i2 < S::MT; ++i2) {
+          const int c0 = 16 * i2 + r, c1 = 16 * i2 + 8 + r;
+          if (2 * t < G) {
+            ob[(2 * t) * D + c0] = o[i2][0] * i0;
+            ob[(2 * t) * D + c1] = o[i2][2] * i0;
           }
-          __syncwarp();
-          i0 += n;
-          const bool last = i0 >= np;
-          // merge states [0, carried + n) into state 0 (or into the outputs when last)
-          merge_states<D>(comb_s, carried + n, STATE, G, lane, last ? nullptr : comb_s,
-                          a.out + ((size_t)b * a.Hq + h * G) * D,
-                          a.lse + (size_t)b * a.Hq + h * G);
-          carried = 1;
+          if (2 * t + 1 < G) {
+            ob[(2 * t + 1) * D + c0] = o[i2][1] * i1;
+            ob[(2 * t + 1) * D + c1] = o[i2][3] * i1;
+          }
+        }
+        if (t == 0 && r < G)
+          a.lse[(size_t)b * a.Hq + h * G + r] =
+              lt > 0.f ? (m_run + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+      } else {
+        const int slot = ua < wa ? 0 : 1;
+        float* my = a.part + ((size_t)gw * 2 + slot) * G * HS;
+#pragma unroll
+        for (int i2 = 0; i2 < S::MT; ++i2) {
+          const int c0 = 16 * i2 + r, c1 = 16 * i2 + 8 + r;
+          if (2 * t < G) {
+            my[(2 * t) * HS + c0] = o[i2][0];
+            my[(2 * t) * HS + c1] = o[i2][2];
+          }
+          if (2 * t + 1 < G) {
+            my[(2 * t + 1) * HS + c0] = o[i2][1];
+            my[(2 * t + 1) * HS + c1] = o[i2][3];
+          }
+        }
+        if (t == 0 && r < G) {
+          my[r * HS + D] = m_run;
+          my[r * HS + D + 1] = lt;
         }
       }
-      if (lane == 0) a.merge_cnt[p] = 0;  // ready for the next call
-      } while (0);
-      // buffer sgi & 1 is free again for segment sgi + 2
-      if (sgi + 2 < n_seg) named_arrive(4 + (sgi & 1), (kConsumers + 1) * 32);
+    };
+
+    for (int j = j0, kc = 0; j < j1; ++j, ++kc) {
+      const int p = u_pair[j];
+      if (p != cur) {
+        if (cur >= 0) finish(cur);
+        cur = p;
+        const int b = p / a.Hkv, h = p % a.Hkv;
+        if (r < G) {
+          const uint4* qrow =
+              reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + h * G + r) * D);
+#pragma unroll
+          for (int jj = 0; jj < S::JQ; ++jj) qa[jj] = qrow[qk_chunk(jj, t)];
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < S::JQ; ++jj) qa[jj] = make_uint4(0, 0, 0, 0);
+        }
+        m_run = -INFINITY;
+        l_run = 0.f;
+#pragma unroll
+        for (int i = 0; i < S::MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+      }
+      const int st = warp + NC * (kc % SPW);
+      bool ok = !*(volatile int*)&abort_flag;
+      if (ok && !mbar_wait(&full_bar[st], (kc / SPW) & 1)) {
+        report(a.status, SA_ERR_TIMEOUT);
+        atomicExch(&abort_flag, 1);
+        ok = false;
+      }
+      const int nv = ok ? u_nv[j] : 0;
+      const uint32_t kbase = stage0 + st * S::STAGE_BYTES;
+      const uint32_t vbase = kbase + S::KV_BYTES;
+      if (nv > 0 && nv < S::CT) {
+        // rows past the valid tokens may hold anything: zero them in V (p = 0 there)
+        uint8_t* vrow = stages + st * S::STAGE_BYTES + S::KV_BYTES;
+        for (int e = lane; e < (S::CT - nv) * S::HALVES * 8; e += 32) {
+          const int row = nv + e / (S::HALVES * 8), cc = e % (S::HALVES * 8);
+          *reinterpret_cast<uint4*>(vrow + (cc >> 3) * S::HALF_BYTES + row * 128 +
+                                    ((cc & 7) << 4)) = make_uint4(0, 0, 0, 0);
+        }
+        // the next TMA copy into this stage must not overtake these plain stores
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+      }
+      if (nv > 0) {
+        // ---- S = Q K^T for 16 tokens (two n-tiles of 8) ----
+        float sc[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+          const int row = nt * 8 + r;
+#pragma unroll
+          for (int jj = 0; jj < S::JQ; ++jj) {
+            const int lc = qk_chunk(jj, t);
+            const uint32_t addr =
+                kbase + (lc >> 3) * S::HALF_BYTES + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
+            const uint4 kv = lds_v4(addr);
+            mma_bf16_16816(sc[nt], qa[jj].x, 0u, qa[jj].y, 0u, kv.x, kv.y);
+            mma_bf16_16816(sc[nt], qa[jj].z, 0u, qa[jj].w, 0u, kv.z, kv.w);
+          }
+        }
+        // ---- online softmax: row = query head r; lane t: tokens 2t,2t+1,8+2t,9+2t ----
+        float x[4];
+        x[0] = 2 * t < nv ? sc[0][0] * a.scale_log2 : -INFINITY;
+        x[1] = 2 * t + 1 < nv ? sc[0][1] * a.scale_log2 : -INFINITY;
+        x[2] = 2 * t + 8 < nv ? sc[1][0] * a.scale_log2 : -INFINITY;
+        x[3] = 2 * t + 9 < nv ? sc[1][1] * a.scale_log2 : -INFINITY;
+        float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+        const float m_new = fmaxf(m_run, mt);  // finite: token 0 of a unit is valid
+        const float alpha = fast_exp2(m_run - m_new);
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - m_new);
+        l_run = l_run * alpha + (pr[0] + pr[1]) + (pr[2] + pr[3]);
+        m_run = m_new;
+        const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * t) * 4);
+        const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) * 4);
+        const uint32_t pb0 = pack_bf16(pr[0], pr[1]);
+        const uint32_t pb1 = pack_bf16(pr[2], pr[3]);
+        // ---- O^T += V^T P^T: m-tile i2 = channels 16 i2 .. 16 i2 + 15 ----
+#pragma unroll
+        for (int i2 = 0; i2 < S::MT; ++i2) {
+          o[i2][0] *= al0;
+          o[i2][1] *= al1;
+          o[i2][2] *= al0;
+          o[i2][3] *= al1;
+          const int lc = 2 * i2 + vsub;
+          const uint32_t addr =
+              vbase + (lc >> 3) * S::HALF_BYTES + vtok * 128 + (((lc & 7) ^ (vtok & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(addr, a0, a1, a2, a3);
+          mma_bf16_16816(o[i2], a0, a1, a2, a3, pb0, pb1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
+    if (cur >= 0) finish(cur);
   }
   __syncthreads();
   if (abort_flag && warp == NC && lane == 0) {
@@ -621,6 +472,103 @@ __global__ void __launch_bounds__((NC + 2) * 32, 1)
   }
 }
 
+// Merge of the pairs cut by warp-range boundaries.  One warp per (pair, query head);
+// lane i holds channels 4i .. 4i+3.  The states of pair p are those of global warps
+// pre[p] / W .. (pre[p+1] - 1) / W, merged in that order with a running maximum.
+struct MergeArgs {
+  const float* part;
+  const int32_t* pre;
+  float* out;
+  float* lse;
+  int n_pairs, G, Hkv, Hq, n_warps;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) attend_merge_kernel(const MergeArgs a) {
+  constexpr int HS = D + 4;
+  constexpr int CH = 8;  // states in flight per lane
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int lane = threadIdx.x & 31;
+  const int wi = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (wi >= a.n_pairs * a.G) return;
+  const int p = wi / a.G, gi = wi % a.G;
+  const int b = p / a.Hkv, h = p % a.Hkv;
+  float* o = a.out + ((size_t)b * a.Hq + h * a.G + gi) * D;
+  float* lse = a.lse + (size_t)b * a.Hq + h * a.G + gi;
+  const int ua = __ldcg(a.pre + p), ub = __ldcg(a.pre + p + 1);
+  const bool on = lane < D / 4;
+  if (ua == ub) {  // nothing selected (empty sequence)
+    if (on) reinterpret_cast<float4*>(o)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0) *lse = -INFINITY;
+    return;
+  }
+  const int total = __ldcg(a.pre + a.n_pairs);
+  const int W = max(1, (total + a.n_warps - 1) / a.n_warps);
+  const int gf = ua / W, gl = (ub - 1) / W;
+  if (gf == gl) return;  // wholly inside one warp's range: written by the attention
+  float m_run = -INFINITY, l_run = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int g0 = gf; g0 <= gl; g0 += CH) {
+    float mk[CH], lk[CH];
+    float4 vk[CH];
+#pragma unroll
+    for (int k = 0; k < CH; ++k) {
+      const int gw = g0 + k;
+      mk[k] = -INFINITY;
+      lk[k] = 0.f;
+      vk[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (gw <= gl) {
+        const int slot = ua < gw * W ? 0 : 1;
+        const float* st = a.part + (((size_t)gw * 2 + slot) * a.G + gi) * HS;
+        mk[k] = __ldcg(st + D);
+        lk[k] = __ldcg(st + D + 1);
+        if (on) vk[k] = __ldcg(reinterpret_cast<const float4*>(st) + lane);
+      }
+    }
+    float mc = m_run;
+#pragma unroll
+    for (int k = 0; k < CH; ++k) mc = fmaxf(mc, mk[k]);
+    if (mc == -INFINITY) continue;  // nothing valid yet
+    const float f = fast_exp2(m_run - mc);  // 0 when m_run = -inf
+    l_run *= f;
+    acc.x *= f;
+    acc.y *= f;
+    acc.z *= f;
+    acc.w *= f;
+#pragma unroll
+    for (int k = 0; k < CH; ++k) {
+      const float w = mk[k] == -INFINITY ? 0.f : fast_exp2(mk[k] - mc);
+      l_run += lk[k] * w;
+      acc.x += vk[k].x * w;
+      acc.y += vk[k].y * w;
+      acc.z += vk[k].z * w;
+      acc.w += vk[k].w * w;
+    }
+    m_run = mc;
+  }
+  const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+  if (on)
+    reinterpret_cast<float4*>(o)[lane] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (lane == 0) *lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+}
+
+static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 template <int D, int P, int NC, int SPW>
 static cudaError_t launch_attend_t(const sa_geom& g, const void* k_cache, const void* v_cache,
                                    AttnArgs a, int n_cta, cudaStream_t stream) {
@@ -629,7 +577,7 @@ static cudaError_t launch_attend_t(const sa_geom& g, const void* k_cache, const 
   const uint64_t rows = (uint64_t)g.n_pool * g.Hkv * P;
   if (!encode_rows_tmap(&kmap, k_cache, D, rows, 64, S::CT)) return cudaErrorInvalidValue;
   if (!encode_rows_tmap(&vmap, v_cache, D, rows, 64, S::CT)) return cudaErrorInvalidValue;
-  const size_t smem = S::smem_bytes(g.Hq / g.Hkv, g.B * g.Hkv);
+  const size_t smem = S::smem_bytes(g.B * g.Hkv);
   static size_t configured = 0;
   if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(attend_gqa_kernel<D, P, NC, SPW>,
@@ -637,45 +585,52 @@ static cudaError_t launch_attend_t(const sa_geom& g, const void* k_cache, const 
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_cta);
-  cfg.blockDim = dim3(S::THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attend_gqa_kernel<D, P, NC, SPW>, kmap, vmap, a);
+  void* args[] = {&kmap, &vmap, &a};
+  cudaError_t e = launch_pdl(reinterpret_cast<const void*>(attend_gqa_kernel<D, P, NC, SPW>),
+                             dim3(n_cta), dim3(S::THREADS), smem, stream, args);
+  if (e != cudaSuccess) return e;
+  MergeArgs m;
+  m.part = a.part;
+  m.pre = a.pre_out;
+  m.out = a.out;
+  m.lse = a.lse;
+  m.n_pairs = g.B * g.Hkv;
+  m.G = g.Hq / g.Hkv;
+  m.Hkv = g.Hkv;
+  m.Hq = g.Hq;
+  m.n_warps = n_cta * NC;
+  void* margs[] = {&m};
+  const int n_tasks = m.n_pairs * m.G;
+  return launch_pdl(reinterpret_cast<const void*>(attend_merge_kernel<D>),
+                    dim3((n_tasks + 3) / 4), dim3(128), 0, stream, margs);
 }
 
-// Pipeline shape: NC consumer warps with SPW units in flight each.  The deepest ring
-// that fits next to the combine area and tables is used.
+// Pipeline shape: kAttnWarps consumer warps with SPW units in flight each; the deepest
+// ring that fits next to the tables is used.
 template <int D, int P>
 static cudaError_t launch_attend_d(const sa_geom& g, const void* k_cache, const void* v_cache,
                                    AttnArgs a, int n_cta, cudaStream_t stream) {
-  const int G = g.Hq / g.Hkv, n_pairs = g.B * g.Hkv;
-  if (AttnShape<D, P, 8, 3>::smem_bytes(G, n_pairs) <= (size_t)kSmemLimit)
-    return launch_attend_t<D, P, 8, 3>(g, k_cache, v_cache, a, n_cta, stream);
-  return launch_attend_t<D, P, 8, 2>(g, k_cache, v_cache, a, n_cta, stream);
+  constexpr int kDeep = D <= 64 ? 4 : 3;
+  if (AttnShape<D, P, kAttnWarps, kDeep>::smem_bytes(g.B * g.Hkv) <= (size_t)kSmemLimit)
+    return launch_attend_t<D, P, kAttnWarps, kDeep>(g, k_cache, v_cache, a, n_cta, stream);
+  return launch_attend_t<D, P, kAttnWarps, 2>(g, k_cache, v_cache, a, n_cta, stream);
 }
 
 int attend_ctas(const sa_geom& g, int K, int sms) {
-  // enough CTAs that no slice exceeds the table capacity even when every pair selects
-  // all K pages
+  // enough CTAs that no CTA's range exceeds the table capacity even when every pair
+  // selects all K pages
   const long long units = (long long)g.B * g.Hkv * K * (g.P / 16);
   const long long need = (units + kMaxUnitsPerCta - 1) / kMaxUnitsPerCta;
   return (int)(need > sms ? need : sms);
 }
 
 size_t attend_partial_floats(const sa_geom& g, int n_cta) {
-  return (size_t)n_cta * 2 * (g.Hq / g.Hkv) * (g.Dv + 4);
+  return (size_t)n_cta * kAttnWarps * 2 * (g.Hq / g.Hkv) * (g.Dv + 4);
 }
 
 bool attend_supported(const sa_geom& g) {
   return g.B * g.Hkv <= kMaxPairs &&
-         AttnShape<128, 16, 8, 2>::smem_bytes(g.Hq / g.Hkv, g.B * g.Hkv) <= (size_t)kSmemLimit;
+         AttnShape<128, 16, kAttnWarps, 2>::smem_bytes(g.B * g.Hkv) <= (size_t)kSmemLimit;
 }
 
 cudaError_t launch_attend(const sa_geom& g, const AttendCall& c, cudaStream_t stream) {
@@ -687,7 +642,7 @@ cudaError_t launch_attend(const sa_geom& g, const AttendCall& c, cudaStream_t st
   a.sel_count = c.sel_count;
   a.sel_phys = c.sel_phys;
   a.part = c.part;
-  a.merge_cnt = c.merge_cnt;
+  a.pre_out = c.pre;
   a.out = c.out;
   a.lse = c.lse;
   a.status = c.status;

@@ -71,8 +71,8 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   off += up256((size_t)g.B * g.Hkv * p.K * 4);
   p.off_arrive = off;
   off += up256((size_t)g.B * g.Hkv * 4);
-  p.off_merge = off;
-  off += up256((size_t)g.B * g.Hkv * 4);
+  p.off_pre = off;
+  off += up256(((size_t)g.B * g.Hkv + 1) * 4);
   p.off_part = off;
   off += up256(attend_partial_floats(g, p.n_cta) * 4);
   p.total = off;
@@ -219,7 +219,7 @@ static int run_attend(const sa_geom& g, const DecodePlan& plan, uint8_t* w, cons
   c.sel_stride = sel_stride;
   c.scale = scale;
   c.part = reinterpret_cast<float*>(w + plan.off_part);
-  c.merge_cnt = reinterpret_cast<uint32_t*>(w + plan.off_merge);
+  c.pre = reinterpret_cast<int32_t*>(w + plan.off_pre);
   c.out = out;
   c.lse = lse;
   c.status = &hdr->status_bits;

@@ -14,7 +14,7 @@ struct DecodePlan {
   int K;      // pages per (sequence, KV head) = budget / P
   int G;      // query heads per KV head
   int n_cta;  // attention CTAs (one per SM, more for very large selections)
-  size_t off_scores, off_sel, off_cnt, off_phys, off_arrive, off_merge, off_part, total;
+  size_t off_scores, off_sel, off_cnt, off_phys, off_arrive, off_pre, off_part, total;
 };
 
 bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan);
@@ -41,8 +41,8 @@ struct AttendCall {
   const int32_t* sel_phys;  // physical pages of sel (nullable: looked up in page_table)
   int sel_stride;
   float scale;
-  float* part;
-  uint32_t* merge_cnt;
+  float* part;     // states of pairs cut by warp-range boundaries
+  int32_t* pre;    // [B*Hkv + 1] pair prefix of units, for the merge kernel
   float* out;
   float* lse;
   int32_t* status;
