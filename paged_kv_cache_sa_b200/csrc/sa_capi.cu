@@ -27,7 +27,8 @@ static int sm_count() {
 
 static bool is_gqa(const sa_geom& g) {
   return !g.v_aliases_k && (g.Dk == 64 || g.Dk == 128) && g.Dv == g.Dk && g.Hq % g.Hkv == 0 &&
-         g.Hq / g.Hkv >= 1 && g.Hq / g.Hkv <= 8 && g.Hkv <= 32 && attend_supported(g);
+         g.Hq / g.Hkv >= 1 && g.Hq / g.Hkv <= 8 && g.Hkv <= 32 && attend_supported(g) &&
+         score_supported(g);
 }
 
 static bool is_latent(const sa_geom& g) {
@@ -60,6 +61,7 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   p.K = budget / g.P;
   p.G = g.Hq / g.Hkv;
   p.n_cta = attend_ctas(g, p.K, sm_count());
+  p.n_score_cta = score_ctas(g, sm_count());
   size_t off = 256;  // status header
   p.off_scores = off;
   off += up256((size_t)g.B * g.Hkv * g.max_pages * 4);
@@ -69,8 +71,6 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   off += up256((size_t)g.B * g.Hkv * 4);
   p.off_phys = off;
   off += up256((size_t)g.B * g.Hkv * p.K * 4);
-  p.off_arrive = off;
-  off += up256((size_t)g.B * g.Hkv * 4);
   p.off_pre = off;
   off += up256(((size_t)g.B * g.Hkv + 1) * 4);
   p.off_part = off;
@@ -197,7 +197,7 @@ static int run_select(const sa_geom& g, const DecodePlan& plan, uint8_t* w, cons
   WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
   return cuda_status(launch_score_select(
       g, q, summ, n_tail > 0 ? k_cache : nullptr, n_tail, page_table, seq_lens, scores,
-      reinterpret_cast<uint32_t*>(w + plan.off_arrive), plan.K, sink / g.P, window / g.P, sel,
+      plan.n_score_cta, plan.K, sink / g.P, window / g.P, sel,
       cnt, phys, &hdr->status_bits, s));
 }
 

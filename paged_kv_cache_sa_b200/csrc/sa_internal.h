@@ -13,8 +13,9 @@ namespace sa {
 struct DecodePlan {
   int K;      // pages per (sequence, KV head) = budget / P
   int G;      // query heads per KV head
-  int n_cta;  // attention CTAs (one per SM, more for very large selections)
-  size_t off_scores, off_sel, off_cnt, off_phys, off_arrive, off_pre, off_part, total;
+  int n_cta;        // attention CTAs (one per SM, more for very large selections)
+  int n_score_cta;  // scoring CTAs (one per SM, more for very long sequences)
+  size_t off_scores, off_sel, off_cnt, off_phys, off_pre, off_part, total;
 };
 
 bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan);
@@ -26,9 +27,12 @@ cudaError_t launch_summaries(const sa_geom& g, const void* k_cache, const int32_
 
 cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
                                 int n_tail, const int32_t* page_table, const int32_t* seq_lens,
-                                float* scores, uint32_t* arrivals, int K, int sink_pages,
+                                float* scores, int n_cta, int K, int sink_pages,
                                 int window_pages, int32_t* sel, int32_t* sel_count,
                                 int32_t* sel_phys, int32_t* status, cudaStream_t stream);
+
+int score_ctas(const sa_geom& g, int sms);
+bool score_supported(const sa_geom& g);
 
 struct AttendCall {
   const void* q;

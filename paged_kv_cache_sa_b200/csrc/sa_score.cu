@@ -1,4 +1,4 @@
-// sa_score.cu -- page scoring (the query-aware page bound) fused with top-k selection.
+// sa_score.cu -- page scoring (the query-aware page bound) and top-k page selection.
 //
 // Method ("SparseEngine" blog, hook-point paragraph: Quest chooses the pages to read at
 // each decode step from the current query; Vortex summary, section 1: hand back the
@@ -8,37 +8,289 @@
 // then per (sequence, KV head) the sink and window pages plus the best remaining pages
 // up to budget/P (equal scores -> lower page index), as an ascending list.
 //
-// Scoring.  Because kmax >= kmin, max(q*kmax, q*kmin) = max(q,0)*kmax + min(q,0)*kmin
-// exactly, so u = [kmin | kmax] . [min(q,0) | max(q,0)], a contraction of length 2*Dk.
-// Every bf16 x bf16 product is exact in fp32; accumulation is fp32.  The G <= 8 query
-// heads are the N=8 side of an m16n8k16 tensor-core tile and 16 pages its M side.
-// A fragments come straight from HBM: each lane reads 16-byte vectors of two summary
-// rows and the contraction's channel order is permuted so that each vector lands in
-// the fragment slots of the lane that loaded it (the query side uses the same order,
-// so the sum is unchanged).  One load instruction covers 64 contiguous bytes of 8 rows,
-// so every sector fetched is used.  The GQA max is a register max + two shuffles.
+// Scoring (score_stream_kernel).  Because kmax >= kmin,
+// max(q*kmax, q*kmin) = max(q,0)*kmax + min(q,0)*kmin exactly, so
+// u = [kmin | kmax] . [min(q,0) | max(q,0)], a contraction of length 2*Dk.  Every
+// bf16 x bf16 product is exact in fp32; accumulation is fp32.  The G <= 8 query heads
+// are the N=8 side of an m16n8k16 tensor-core tile and 16 pages its M side.
+// The work is a flattened list of tiles (sequence, head group, 16 consecutive pages);
+// each persistent CTA takes a contiguous slice.  A producer warp gathers each tile
+// through the page table with one bulk copy per page (the page's summaries of the
+// head group are contiguous) plus one for the group's query rows, into a ring of
+// shared-memory stages; consumer warps (one per KV head of the group) read A and B
+// fragments with 16-byte shared loads in a permuted channel order (the query side uses
+// the same order, so the sum is unchanged) -- page slots are padded by 64 bytes so
+// those loads are free of bank conflicts -- and write the GQA-max score row.
+// HBM-bound: bytes per (page, KV head) = 2 * Dk * 2 (summary) + 4 / Hkv (page table).
 //
-// Decode-time summary refresh.  When asked, the warp whose 16-page tile holds a
-// sequence's newest page first recomputes that page's min/max from K (the page that
-// received the appended token) and scores the fresh summary.
-//
-// Selection.  Each CTA scores 128 pages of one (sequence, KV head); the last CTA to
-// finish for that pair (an atomic arrival counter, no waiting) turns the scores into
-// order-preserving 32-bit keys in shared memory (forced pages get key 0, below every
-// real score) and runs an MSB-first 8-bit radix select (4 passes, warp-aggregated
+// Selection (select_kernel, one CTA per (sequence, KV head), launched programmatically
+// dependent on the scoring grid).  Before waiting for the scores it recomputes the
+// summaries of the sequence's newest pages from K when asked (the pages that received
+// appended tokens) and scores them; those scores replace the streamed ones, so the
+// scoring grid may read either version of those summaries.  Then it turns the scores
+// into order-preserving 32-bit keys in shared memory (forced pages get key 0, below
+// every real score) and runs an MSB-first 8-bit radix select (warp-aggregated
 // shared-memory histograms, one warp scans the 256 bins).  That gives the exact key T
 // of the k-th best candidate and how many keys equal to T are needed; a final pass
 // marks forced pages, keys > T and the lowest-index keys == T, and two block scans
-// write the ascending list.  Deterministic.  HBM-bound: bytes per (page, KV head) =
-// 2 * Dk * 2 (summary) + 4 (page-table entry).
+// write the ascending list.  Deterministic.
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
 namespace sa {
 
-constexpr int kScoreWarps = 8;
-constexpr int kScoreThreads = kScoreWarps * 32;
-constexpr int kPagesPerCta = 16 * kScoreWarps;
+constexpr int kTilePages = 16;  // pages per tile: the M side of one MMA
+constexpr int kScoreConsumers = 8;
+constexpr int kScoreThreads = (kScoreConsumers + 1) * 32;
+constexpr int kMaxTilesPerCta = 128;
+constexpr int kSlotPad = 64;  // odd multiple of 64 B between page slots: no bank conflicts
+constexpr int kSelectThreads = 256;
+constexpr int kScoreSmemLimit = 227 * 1024;
+
+struct ScoreArgs {
+  const uint16_t* q;
+  const uint8_t* summ;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  float* scores;  // [B][Hkv][max_pages]
+  int32_t* status;
+  int B, Hq, Hkv, G, P, max_pages, n_pool;
+  int HG, n_hg, WPS, NST;              // heads per tile, head groups, warp groups, stages
+  int slot_bytes, q_off, stage_bytes;  // stage: [16][slot_bytes] page slots | q rows
+};
+
+__device__ __forceinline__ void named_barrier_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// the sequence owning flattened tile u: largest b with pre[b] <= u
+__device__ __forceinline__ int find_seq(const int* pre, int n, int u) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= u)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const ScoreArgs a) {
+  constexpr int J = D / 16;  // 16-byte chunks per lane of the 2*D-long contraction row
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stages = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  int* pre = reinterpret_cast<int*>(stages + (size_t)a.NST * a.stage_bytes);  // [B + 1]
+  int* ptab = pre + a.B + 1;                       // [kMaxTilesPerCta * 16]
+  int* t_b = ptab + kMaxTilesPerCta * kTilePages;  // per tile of the slice
+  int* t_hg = t_b + kMaxTilesPerCta;
+  int* t_p0 = t_hg + kMaxTilesPerCta;
+  int* t_np = t_p0 + kMaxTilesPerCta;  // pages in the tile
+  int* t_vm = t_np + kMaxTilesPerCta;  // mask of pages with a valid slot
+  __shared__ __align__(8) uint64_t full_bar[8];
+  __shared__ __align__(8) uint64_t empty_bar[8];
+  __shared__ int sh_nt, abort_flag;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = blockIdx.x, n_cta = gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < a.NST; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], a.HG);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // everything read below may come from the previous kernel of the stream
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+
+  if (warp == kScoreConsumers) {
+    // ===================== producer warp: tables =====================
+    // 1. tiles per sequence: n_hg * ceil(pages / 16), prefix-summed
+    int carry = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      int n = 0;
+      if (b < a.B) {
+        const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
+        const int nb = (L + a.P - 1) / a.P;
+        n = a.n_hg * ((nb + kTilePages - 1) / kTilePages);
+      }
+      int incl = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (b < a.B) pre[b] = carry + incl - n;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) pre[a.B] = carry;
+    __syncwarp();
+    const int total = carry;
+    const int W = max(1, (total + n_cta - 1) / n_cta);
+    const int T0 = min(total, c * W);
+    const int nt = min(total, T0 + W) - T0;  // <= kMaxTilesPerCta (the host sizes the grid)
+    // 2. the slice's tiles: sequence, head group, first page, page count
+    for (int i = lane; i < nt; i += 32) {
+      const int u = T0 + i;
+      const int b = find_seq(pre, a.B, u);
+      const int ntb = (pre[b + 1] - pre[b]) / a.n_hg;  // tiles per head group
+      const int rem = u - pre[b];
+      const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
+      const int nb = (L + a.P - 1) / a.P;
+      t_b[i] = b;
+      t_hg[i] = rem / ntb;
+      t_p0[i] = (rem % ntb) * kTilePages;
+      t_np[i] = min(kTilePages, nb - (rem % ntb) * kTilePages);
+    }
+    __syncwarp();
+    // 3. page-table entries of the slice (16 loads in flight per lane)
+    const int ne = nt * kTilePages;
+    for (int e0 = 0; e0 < ne; e0 += 32 * 16) {
+      int v[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int e = e0 + 32 * k + lane;
+        v[k] = -1;
+        if (e < ne) {
+          const int i = e >> 4, pg = e & 15;
+          if (pg < t_np[i]) v[k] = a.page_table[(size_t)t_b[i] * a.max_pages + t_p0[i] + pg];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int e = e0 + 32 * k + lane;
+        if (e < ne) ptab[e] = v[k];
+      }
+    }
+    __syncwarp();
+    for (int i = lane; i < nt; i += 32) {
+      int vm = 0;
+      for (int pg = 0; pg < t_np[i]; ++pg) {
+        const int ph = ptab[i * kTilePages + pg];
+        if (ph >= 0 && ph < a.n_pool)
+          vm |= 1 << pg;
+        else
+          report(a.status, SA_ERR_DEVICE_CHECK);
+      }
+      t_vm[i] = vm;
+    }
+    if (lane == 0) sh_nt = nt;
+    __syncwarp();
+    named_barrier_sync(1, kScoreThreads);  // tables ready
+
+    // ===================== producer warp: bulk-copy issue =====================
+    const uint32_t slot_data = (uint32_t)a.HG * 4 * D;  // one page's summaries of the group
+    const uint32_t q_bytes = (uint32_t)a.HG * a.G * D * 2;
+    uint64_t t_idle = 0;
+    for (int k = 0; k < nt;) {
+      const int s = k % a.NST;
+      bool ready = k < a.NST;
+      if (!ready && lane == 0) ready = mbar_test(&empty_bar[s], ((k / a.NST) - 1) & 1);
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) {
+        const uint64_t now = global_ns();
+        if (t_idle == 0) t_idle = now;
+        const int to = (now - t_idle > kWaitLimitNs) || *(volatile int*)&abort_flag;
+        if (__shfl_sync(0xffffffffu, to, 0)) {
+          if (lane == 0) {
+            report(a.status, SA_ERR_TIMEOUT);
+            atomicExch(&abort_flag, 1);
+          }
+          break;
+        }
+        continue;
+      }
+      t_idle = 0;
+      const int vm = t_vm[k], b = t_b[k], hg = t_hg[k];
+      uint8_t* st = stages + (size_t)s * a.stage_bytes;
+      if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], __popc(vm) * slot_data + q_bytes);
+      __syncwarp();
+      if (lane < kTilePages && ((vm >> lane) & 1)) {
+        const int ph = ptab[k * kTilePages + lane];
+        bulk_load(st + lane * a.slot_bytes, a.summ + ((size_t)ph * a.Hkv + hg * a.HG) * 4 * D,
+                  slot_data, &full_bar[s]);
+      } else if (lane == kTilePages) {
+        bulk_load(st + a.q_off, a.q + ((size_t)b * a.Hq + (size_t)hg * a.HG * a.G) * D, q_bytes,
+                  &full_bar[s]);
+      }
+      ++k;
+    }
+  } else {
+    // ===================== consumer warps =====================
+    named_barrier_sync(1, kScoreThreads);  // tables ready
+    const int r = lane >> 2, t = lane & 3;
+    const int grp = warp / a.HG, hh = warp % a.HG;  // stage group, head within the group
+    const int nt = sh_nt;
+    const bool v0 = 2 * t < a.G, v1 = 2 * t + 1 < a.G;
+    for (int k = grp; k < nt; k += a.WPS) {
+      const int s = k % a.NST;
+      bool ok = !*(volatile int*)&abort_flag;
+      if (ok && !mbar_wait(&full_bar[s], (k / a.NST) & 1)) {
+        report(a.status, SA_ERR_TIMEOUT);
+        atomicExch(&abort_flag, 1);
+        ok = false;
+      }
+      if (ok) {
+        const int b = t_b[k], h = t_hg[k] * a.HG + hh, p0 = t_p0[k], np = t_np[k];
+        const int vm = t_vm[k];
+        const uint32_t st = smem_u32(stages + (size_t)s * a.stage_bytes);
+        // B: [min(q,0) | max(q,0)] of query head n = r of KV head h, chunk 4j + t
+        uint32_t bq[J][4];
+        const uint32_t qrow = st + a.q_off + (uint32_t)(hh * a.G + (r < a.G ? r : 0)) * D * 2;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const int cc = 4 * j + t;  // chunk of the 2D-long contraction
+          const uint4 v = lds_v4(qrow + (cc % (D / 8)) * 16);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t neg = ((w[e] >> 15) & 0x00010001u) * 0xFFFFu;  // negative halves
+            bq[j][e] = r < a.G ? ((cc < D / 8) ? (w[e] & neg) : (w[e] & ~neg)) : 0u;
+          }
+        }
+        // A: rows r and r + 8 of the tile (pages p0 + r, p0 + r + 8)
+        const bool va = (vm >> r) & 1, vb = (vm >> (r + 8)) & 1;
+        const uint32_t rowa = st + r * a.slot_bytes + hh * 4 * D;
+        const uint32_t rowb = rowa + 8 * a.slot_bytes;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const uint4 ra = va ? lds_v4(rowa + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
+          const uint4 rb = vb ? lds_v4(rowb + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
+          mma_bf16_16816(acc, ra.x, rb.x, ra.y, rb.y, bq[j][0], bq[j][1]);
+          mma_bf16_16816(acc, ra.z, rb.z, ra.w, rb.w, bq[j][2], bq[j][3]);
+        }
+        // acc: [page r][heads 2t, 2t+1], [page r+8][heads 2t, 2t+1]
+        float m0 = fmaxf(v0 ? acc[0] : -INFINITY, v1 ? acc[1] : -INFINITY);
+        float m1 = fmaxf(v0 ? acc[2] : -INFINITY, v1 ? acc[3] : -INFINITY);
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+        if (t == 0) {
+          float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages + p0;
+          if (r < np) srow[r] = m0;
+          if (r + 8 < np) srow[r + 8] = m1;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+    }
+  }
+  __syncthreads();
+  if (abort_flag && warp == kScoreConsumers && lane == 0) {
+    // a wait expired: give copies still in flight a bounded time (10 ms) to land
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < 10000000ull) {
+    }
+  }
+}
 
 template <int NT>
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total) {
@@ -69,118 +321,25 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total)
   return res;
 }
 
-// Radix select of one (sequence, KV head) by the whole CTA; see the file comment.
-template <int NT>
-__device__ void block_select(const float* srow, int nb, int K, int s_pages, int w_pages,
-                             uint32_t* keys, int32_t* out, int32_t* cnt_out,
-                             const int32_t* ptab, int32_t* phys_out) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t sh_bin, sh_above;
-  __shared__ int warp_tot[NT / 32 + 1];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (nb <= K) {
-    for (int i = tid; i < K; i += NT) {
-      out[i] = i < nb ? i : -1;
-      if (phys_out) phys_out[i] = i < nb ? ptab[i] : -1;
-    }
-    if (tid == 0) *cnt_out = nb;
-    return;
-  }
-  const int wbeg = nb - w_pages;
-  for (int p = tid; p < nb; p += NT)
-    keys[p] = (p < s_pages || p >= wbeg) ? 0u : f32_order_key(__ldcg(srow + p));
-  __syncthreads();
-
-  uint32_t prefix = 0, pmask = 0;
-  int k_rem = K - s_pages - w_pages;     // < number of candidates here
-  if (k_rem == 0) prefix = 0xFFFFFFFFu;  // forced pages only: no key reaches T
-#pragma unroll 1
-  for (int shift = 24; shift >= 0 && k_rem > 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) hist[i] = 0;
-    __syncthreads();
-    for (int p = tid; p < nb; p += NT) {
-      const uint32_t key = keys[p];
-      if ((key & pmask) == prefix) {
-        const uint32_t bin = (key >> shift) & 255u;
-        const unsigned act = __activemask();
-        const unsigned peers = __match_any_sync(act, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-      }
-    }
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t c[8], tot = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c[i] = hist[lane * 8 + i];
-        tot += c[i];
-      }
-      uint32_t incl = tot;  // keys in bins of lanes >= this lane
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t u = __shfl_down_sync(0xffffffffu, incl, off);
-        if (lane + off < 32) incl += u;
-      }
-      uint32_t run = incl - tot;  // keys in higher bins than this lane's
-#pragma unroll
-      for (int i = 7; i >= 0; --i) {
-        if (run < (uint32_t)k_rem && run + c[i] >= (uint32_t)k_rem) {
-          sh_bin = lane * 8 + i;
-          sh_above = run;
-        }
-        run += c[i];
-      }
-    }
-    __syncthreads();
-    prefix |= sh_bin << shift;
-    pmask |= 255u << shift;
-    k_rem -= (int)sh_above;
-    __syncthreads();
-  }
-  const uint32_t T = prefix;
-
-  const int seg = (nb + NT - 1) / NT;
-  const int beg = min(nb, tid * seg), end = min(nb, beg + seg);
-  int n_eq = 0;
-  for (int p = beg; p < end; ++p) n_eq += keys[p] == T;
-  int tot;
-  const int eq_rank = block_excl_scan<NT>(n_eq, warp_tot, &tot);
-  int n_sel = 0;
-  for (int p = beg, er = eq_rank; p < end; ++p) {
-    const uint32_t key = keys[p];
-    const bool is_eq = key == T;
-    n_sel += (p < s_pages || p >= wbeg) || key > T || (is_eq && er < k_rem);
-    er += is_eq;
-  }
-  int pos = block_excl_scan<NT>(n_sel, warp_tot, &tot);
-  for (int p = beg, er = eq_rank; p < end; ++p) {
-    const uint32_t key = keys[p];
-    const bool is_eq = key == T;
-    if ((p < s_pages || p >= wbeg) || key > T || (is_eq && er < k_rem)) {
-      out[pos] = p;
-      if (phys_out) phys_out[pos] = ptab[p];
-      ++pos;
-    }
-    er += is_eq;
-  }
-  for (int i = tot + tid; i < K; i += NT) {
-    out[i] = -1;
-    if (phys_out) phys_out[i] = -1;
-  }
-  if (tid == 0) *cnt_out = tot;
-}
-
-// Recompute the summary of one (physical page, KV head) from K (one warp).
+// Recompute the summary of one (physical page, KV head) from K (one warp), store it,
+// and return in every lane its score for the G query heads at qh (max over heads).
 template <int D>
-__device__ __forceinline__ void warp_refresh_summary(const uint4* __restrict__ k_cache,
-                                                     uint4* __restrict__ summ, int phys, int h,
-                                                     int Hkv, int P, int valid, int lane) {
+__device__ float warp_refresh_and_score(const uint4* __restrict__ k_cache,
+                                        uint4* __restrict__ summ, const uint16_t* qh, int G,
+                                        int phys, int h, int Hkv, int P, int valid, int lane) {
   constexpr int CPR = D / 8;     // 8 or 16 chunks per row
   constexpr int RPI = 32 / CPR;  // rows per warp iteration
   const int c = lane % CPR;
   const uint4* blk = k_cache + ((size_t)phys * Hkv + h) * P * CPR;
   uint4 mn = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
   uint4 mx = make_uint4(0x80008000u, 0x80008000u, 0x80008000u, 0x80008000u);
+  // query rows first: independent of K, so their loads are in flight with K's
+  uint4 qv[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g)
+    qv[g] = (g < G && lane < CPR) ? *reinterpret_cast<const uint4*>(qh + (size_t)g * D + c * 8)
+                                  : make_uint4(0, 0, 0, 0);
+#pragma unroll 4
   for (int t = lane / CPR; t < valid; t += RPI) {
     const uint4 v = __ldcg(blk + (size_t)t * CPR + c);
     const uint32_t k0 = bf2_key(v.x), k1 = bf2_key(v.y), k2 = bf2_key(v.z), k3 = bf2_key(v.w);
@@ -200,204 +359,293 @@ __device__ __forceinline__ void warp_refresh_summary(const uint4* __restrict__ k
     mx.z = __vmaxs2(mx.z, __shfl_xor_sync(0xffffffffu, mx.z, off));
     mx.w = __vmaxs2(mx.w, __shfl_xor_sync(0xffffffffu, mx.w, off));
   }
+  const uint4 kmin = make_uint4(bf2_key(mn.x), bf2_key(mn.y), bf2_key(mn.z), bf2_key(mn.w));
+  const uint4 kmax = make_uint4(bf2_key(mx.x), bf2_key(mx.y), bf2_key(mx.z), bf2_key(mx.w));
   uint4* out = summ + ((size_t)phys * Hkv + h) * 2 * CPR;
   if (lane < CPR) {
-    __stcg(out + c, make_uint4(bf2_key(mn.x), bf2_key(mn.y), bf2_key(mn.z), bf2_key(mn.w)));
-    __stcg(out + CPR + c, make_uint4(bf2_key(mx.x), bf2_key(mx.y), bf2_key(mx.z), bf2_key(mx.w)));
+    __stcg(out + c, kmin);
+    __stcg(out + CPR + c, kmax);
   }
+  const uint32_t lo[4] = {kmin.x, kmin.y, kmin.z, kmin.w};
+  const uint32_t hi[4] = {kmax.x, kmax.y, kmax.z, kmax.w};
+  float best = -INFINITY;
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    if (g >= G) break;
+    const uint32_t qw[4] = {qv[g].x, qv[g].y, qv[g].z, qv[g].w};
+    float part = 0.f;
+    if (lane < CPR) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const float qf = __uint_as_float(hf ? (qw[e] & 0xFFFF0000u) : (qw[e] << 16));
+          const float a0 = __uint_as_float(hf ? (lo[e] & 0xFFFF0000u) : (lo[e] << 16));
+          const float a1 = __uint_as_float(hf ? (hi[e] & 0xFFFF0000u) : (hi[e] << 16));
+          part += fmaxf(qf * a1, qf * a0);
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    best = fmaxf(best, part);
+  }
+  return best;
 }
 
-struct ScoreArgs {
+constexpr int kMaxTail = 16;
+constexpr int kHistBits = 11;  // digit of the one-pass histogram
+constexpr int kHistBins = 1 << kHistBits;
+constexpr int kBinCap = 256;             // boundary-bin size ranked exactly
+constexpr uint32_t kWin = 0xFFFFFFFFu;   // marks a candidate taken from the boundary bin
+
+struct SelectArgs {
   const uint16_t* q;
   uint4* summ;
-  const uint4* k_cache;  // non-null: refresh the last n_tail pages' summaries first
+  const uint4* k_cache;  // non-null: refresh the newest n_tail pages' summaries first
   const int32_t* page_table;
   const int32_t* seq_lens;
   float* scores;       // [B][Hkv][max_pages]
-  uint32_t* arrivals;  // [B][Hkv] CTA arrival counters (zero between calls)
   int32_t* sel;        // [B][Hkv][K]
   int32_t* sel_count;  // [B][Hkv]
   int32_t* sel_phys;   // [B][Hkv][K] physical pages of the selection (nullable)
   int32_t* status;
   int Hq, Hkv, P, max_pages, n_pool, K, s_pages, w_pages, n_tail;
+  int ptab_in_smem;  // the sequence's page-table row is staged next to the keys
 };
 
 template <int D>
-__global__ void __launch_bounds__(kScoreThreads) score_select_kernel(const ScoreArgs a) {
-  constexpr int NCH = 2 * D / 8;      // 16-byte chunks per summary row [kmin | kmax]
-  constexpr int J = NCH / 4;          // chunks per lane per row
-  extern __shared__ uint32_t keys[];  // [max_pages], used by the selecting CTA only
-  __shared__ int is_last;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r = lane >> 2, t = lane & 3;
-  const int h = blockIdx.x % a.Hkv, tile = blockIdx.x / a.Hkv, b = blockIdx.y;
+__global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs a) {
+  constexpr int NT = kSelectThreads;
+  extern __shared__ uint32_t keys[];  // [max_pages] keys, then [max_pages] page table
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ uint32_t sh_bin, sh_above, red[2 * (NT / 32)];
+  __shared__ uint32_t bin_key[kBinCap];
+  __shared__ int bin_page[kBinCap];
+  __shared__ int warp_tot[NT / 32 + 1], sh_n;
+  __shared__ float tail_score[kMaxTail];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int G = a.Hq / a.Hkv;
+  // The scoring grid passed its own wait before letting this grid start, so the
+  // inputs of the call (everything but the scores) are complete here.
   const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
   const int nb = (L + a.P - 1) / a.P;
-  const int ntiles = max(1, (nb + kPagesPerCta - 1) / kPagesPerCta);
+  const int32_t* ptab_g = a.page_table + (size_t)b * a.max_pages;
   float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages;
-
-  // the previous kernel of the stream may still be using this workspace
+  const int tail0 = max(0, nb - a.n_tail);
+  const int n_tail = a.k_cache ? nb - tail0 : 0;
+  // 1. decode-time refresh of the newest pages (overlaps the scoring grid)
+  for (int i = warp; i < n_tail; i += NT / 32) {
+    const int lp = tail0 + i;
+    const int ph = ptab_g[lp];
+    float sc = 0.f;
+    if (ph >= 0 && ph < a.n_pool)
+      sc = warp_refresh_and_score<D>(a.k_cache, a.summ, a.q + ((size_t)b * a.Hq + h * G) * D,
+                                     G, ph, h, a.Hkv, a.P, min(a.P, L - lp * a.P), lane);
+    if (lane == 0) tail_score[i] = sc;
+  }
+  // 2. wait for the scores
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // let the attention kernel get launched; it waits for this grid before reading
   asm volatile("griddepcontrol.launch_dependents;");
-
-  const int p0 = tile * kPagesPerCta + warp * 16;
-  if (tile >= ntiles) {  // past the sequence: scores are -inf there
-    if (lane < 16 && p0 + lane < a.max_pages) srow[p0 + lane] = -INFINITY;
+  __syncthreads();
+  int32_t* out = a.sel + ((size_t)b * a.Hkv + h) * a.K;
+  int32_t* cnt_out = a.sel_count + (size_t)b * a.Hkv + h;
+  int32_t* phys_out = a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.K : nullptr;
+  for (int i = tid; i < n_tail; i += NT) srow[tail0 + i] = tail_score[i];
+  for (int p = nb + tid; p < a.max_pages; p += NT) srow[p] = -INFINITY;
+  const int K = a.K;
+  if (nb <= K) {  // everything fits the budget
+    for (int i = tid; i < K; i += NT) {
+      out[i] = i < nb ? i : -1;
+      if (phys_out) phys_out[i] = i < nb ? ptab_g[i] : -1;
+    }
+    if (tid == 0) *cnt_out = nb;
     return;
   }
-
-  if (p0 < a.max_pages) {
-    // decode-time refresh of the newest pages' summaries that fall in this warp's tile
-    bool refreshed = false;
-    if (a.k_cache) {
-      for (int lp = max(p0, nb - a.n_tail); lp < min(p0 + 16, nb); ++lp) {
-        const int ph = a.page_table[(size_t)b * a.max_pages + lp];
-        if (ph < 0 || ph >= a.n_pool) continue;
-        warp_refresh_summary<D>(a.k_cache, a.summ, ph, h, a.Hkv, a.P, min(a.P, L - lp * a.P),
-                                lane);
-        refreshed = true;
-      }
-      if (refreshed) {
-        __threadfence_block();
-        __syncwarp();
-      }
-    }
-
-    // A: summary rows of pages p0 + r and p0 + r + 8 (chunk 4j + t of each row)
-    const int pa = p0 + r, pb = p0 + r + 8;
-    uint4 ra[J], rb[J];
-    {
-      const int pha = pa < nb ? a.page_table[(size_t)b * a.max_pages + pa] : 0;
-      const int phb = pb < nb ? a.page_table[(size_t)b * a.max_pages + pb] : 0;
-      if ((pha < 0 || pha >= a.n_pool || phb < 0 || phb >= a.n_pool) && t == 0)
-        report(a.status, SA_ERR_DEVICE_CHECK);
-      const uint4* rowa = (pa < nb && pha >= 0 && pha < a.n_pool)
-                              ? a.summ + ((size_t)pha * a.Hkv + h) * NCH
-                              : nullptr;
-      const uint4* rowb = (pb < nb && phb >= 0 && phb < a.n_pool)
-                              ? a.summ + ((size_t)phb * a.Hkv + h) * NCH
-                              : nullptr;
-      if (refreshed) {  // rows just written by this warp: read them through L2
+  int32_t* ptab_s = a.ptab_in_smem ? reinterpret_cast<int32_t*>(keys + a.max_pages) : nullptr;
+  // 3. keys (8 loads in flight per thread) and the candidates' key range
+  const int wbeg = nb - a.w_pages;
+  uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+  for (int p0 = 0; p0 < nb; p0 += NT * 8) {
+    float v[8];
+    int pt[8];
 #pragma unroll
-        for (int j = 0; j < J; ++j) {
-          ra[j] = rowa ? __ldcg(rowa + 4 * j + t) : make_uint4(0, 0, 0, 0);
-          rb[j] = rowb ? __ldcg(rowb + 4 * j + t) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < 8; ++k) {
+      const int p = p0 + k * NT + tid;
+      v[k] = p < nb ? __ldcg(srow + p) : 0.f;
+      pt[k] = (ptab_s && p < nb) ? ptab_g[p] : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int p = p0 + k * NT + tid;
+      if (p < nb) {
+        const float sv = (n_tail > 0 && p >= tail0) ? tail_score[p - tail0] : v[k];
+        const bool forced = p < a.s_pages || p >= wbeg;
+        const uint32_t key = forced ? 0u : f32_order_key(sv);
+        keys[p] = key;
+        if (!forced) {
+          kmn = min(kmn, key);
+          kmx = max(kmx, key);
         }
-      } else {
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-          ra[j] = rowa ? ldg_nc_v4(rowa + 4 * j + t) : make_uint4(0, 0, 0, 0);
-          rb[j] = rowb ? ldg_nc_v4(rowb + 4 * j + t) : make_uint4(0, 0, 0, 0);
-        }
+        if (ptab_s) ptab_s[p] = pt[k];
       }
     }
+  }
+  kmn = __reduce_min_sync(0xffffffffu, kmn);
+  kmx = __reduce_max_sync(0xffffffffu, kmx);
+  if (lane == 0) {
+    red[warp] = kmn;
+    red[NT / 32 + warp] = kmx;
+  }
+  __syncthreads();
+  kmn = 0xFFFFFFFFu;
+  kmx = 0u;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    kmn = min(kmn, red[w]);
+    kmx = max(kmx, red[NT / 32 + w]);
+  }
 
-    // B: [min(q,0) | max(q,0)] of query head n = r of the group, same chunk order
-    uint4 bq[J];
-    if (r < G) {
-      const uint4* qrow =
-          reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + h * G + r) * D);
-#pragma unroll
-      for (int j = 0; j < J; ++j) {
-        const int c = 4 * j + t;  // chunk of the 2D-long contraction
-        const uint4 v = qrow[c % (D / 8)];
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t neg = ((w[e] >> 15) & 0x00010001u) * 0xFFFFu;  // negative halves
-          w[e] = (c < D / 8) ? (w[e] & neg) : (w[e] & ~neg);
-        }
-        bq[j] = make_uint4(w[0], w[1], w[2], w[3]);
+  // 4. threshold: a candidate is taken when its key >= thr or it was marked kWin.
+  // MSB-first radix select with 11-bit digits starting at the highest bit in which the
+  // candidates differ (the bits above are common to all of them); it stops as soon as
+  // the boundary bin is wholly taken or small enough to rank exactly.
+  const int k_rem0 = K - a.s_pages - a.w_pages;  // < number of candidates here
+  uint64_t thr = 1ull << 32;                      // above every key: forced pages only
+  if (k_rem0 > 0) {
+    const uint32_t diff = kmn ^ kmx;
+    int hi = diff ? 31 - __clz(diff) : -1;  // highest undecided bit
+    uint32_t pmask;                         // bits decided so far (above hi)
+    if (hi < 0)
+      pmask = 0xFFFFFFFFu;  // all candidates are equal
+    else if (hi == 31)
+      pmask = 0u;
+    else
+      pmask = ~((2u << hi) - 1u);
+    uint32_t pval = kmn & pmask;
+    int k_need = k_rem0;
+    int state = 0;  // 0: go on, 1: thr set, 2: tie on the full key
+    while (state == 0) {
+      if (hi < 0) {
+        state = 2;
+        break;
       }
-    } else {
+      const int lo = max(0, hi - (kHistBits - 1));
+      const uint32_t dmask = (2u << (hi - lo)) - 1u;
+      for (int i = tid; i < kHistBins; i += NT) hist[i] = 0;
+      __syncthreads();
+      for (int p = tid; p < nb; p += NT) {
+        const uint32_t key = keys[p];
+        if (!(p < a.s_pages || p >= wbeg) && (key & pmask) == pval)
+          atomicAdd(&hist[(key >> lo) & dmask], 1u);
+      }
+      __syncthreads();
+      // bins owned 8 per thread; candidates in bins above each thread's range
+      constexpr int BPT = kHistBins / NT;
+      int mine = 0;
 #pragma unroll
-      for (int j = 0; j < J; ++j) bq[j] = make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < BPT; ++i) mine += hist[tid * BPT + i];
+      int total;
+      const int below = block_excl_scan<NT>(mine, warp_tot, &total);
+      int run = total - below - mine;
+      for (int i = BPT - 1; i >= 0; --i) {
+        const int cnt = hist[tid * BPT + i];
+        if (run < k_need && run + cnt >= k_need) {
+          sh_bin = tid * BPT + i;
+          sh_above = run;
+        }
+        run += cnt;
+      }
+      __syncthreads();
+      const uint32_t bstar = sh_bin;
+      k_need -= (int)sh_above;
+      const int nbin = hist[bstar];
+      pval |= bstar << lo;
+      pmask |= dmask << lo;
+      if (nbin == k_need) {  // the whole boundary bin is taken
+        thr = pval;
+        state = 1;
+      } else if (nbin <= kBinCap) {
+        // exact ranking inside the boundary bin: larger key first, then lower page
+        if (tid == 0) sh_n = 0;
+        __syncthreads();
+        for (int p = tid; p < nb; p += NT) {
+          const uint32_t key = keys[p];
+          if (!(p < a.s_pages || p >= wbeg) && (key & pmask) == pval) {
+            const int i = atomicAdd(&sh_n, 1);
+            bin_key[i] = key;
+            bin_page[i] = p;
+          }
+        }
+        __syncthreads();
+        if (tid < nbin) {
+          const uint32_t key = bin_key[tid];
+          const int pg = bin_page[tid];
+          int rank = 0;
+          for (int j = 0; j < nbin; ++j) {
+            const uint32_t kj = bin_key[j];
+            rank += kj > key || (kj == key && bin_page[j] < pg);
+          }
+          if (rank < k_need) keys[pg] = kWin;
+        }
+        thr = (uint64_t)pval + (1ull << lo);
+        state = 1;
+      }
+      hi = lo - 1;
+      __syncthreads();
     }
-
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      mma_bf16_16816(acc, ra[j].x, rb[j].x, ra[j].y, rb[j].y, bq[j].x, bq[j].y);
-      mma_bf16_16816(acc, ra[j].z, rb[j].z, ra[j].w, rb[j].w, bq[j].z, bq[j].w);
-    }
-    // acc: [page r][heads 2t, 2t+1], [page r+8][heads 2t, 2t+1]
-    const bool v0 = 2 * t < G, v1 = 2 * t + 1 < G;
-    float m0 = fmaxf(v0 ? acc[0] : -INFINITY, v1 ? acc[1] : -INFINITY);
-    float m1 = fmaxf(v0 ? acc[2] : -INFINITY, v1 ? acc[3] : -INFINITY);
-    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
-    if (t == 0) {
-      if (pa < a.max_pages) srow[pa] = pa < nb ? m0 : -INFINITY;
-      if (pb < a.max_pages) srow[pb] = pb < nb ? m1 : -INFINITY;
+    if (state == 2) {
+      // the boundary keys are all equal to T = pval: take the lowest-index ones
+      const uint32_t T = pval;
+      const int seg = (nb + NT - 1) / NT;
+      const int beg = min(nb, tid * seg), end = min(nb, beg + seg);
+      int n_eq = 0;
+      for (int p = beg; p < end; ++p) n_eq += !(p < a.s_pages || p >= wbeg) && keys[p] == T;
+      int tot;
+      int er = block_excl_scan<NT>(n_eq, warp_tot, &tot);
+      for (int p = beg; p < end; ++p) {
+        if (!(p < a.s_pages || p >= wbeg) && keys[p] == T) {
+          if (er < k_need) keys[p] = kWin;
+          ++er;
+        }
+      }
+      thr = (uint64_t)T + 1;
+      __syncthreads();
     }
   }
 
-  // ---- arrival: the last CTA of this (sequence, KV head) selects ----
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t* cnt = a.arrivals + (size_t)b * a.Hkv + h;
-    const uint32_t old = atomicAdd(cnt, 1u);
-    is_last = old == (uint32_t)(ntiles - 1);
-    if (is_last) *cnt = 0;  // ready for the next call
+  // 5. ascending list: forced pages and taken candidates
+  const int seg = (nb + NT - 1) / NT;
+  const int beg = min(nb, tid * seg), end = min(nb, beg + seg);
+  auto taken = [&](int p) {
+    if (p < a.s_pages || p >= wbeg) return true;
+    const uint32_t key = keys[p];
+    return key == kWin || (uint64_t)key >= thr;
+  };
+  int n_sel = 0;
+  for (int p = beg; p < end; ++p) n_sel += taken(p);
+  int tot;
+  int pos = block_excl_scan<NT>(n_sel, warp_tot, &tot);
+  for (int p = beg; p < end; ++p) {
+    if (taken(p)) {
+      out[pos] = p;
+      if (phys_out) phys_out[pos] = ptab_s ? ptab_s[p] : ptab_g[p];
+      ++pos;
+    }
   }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  block_select<kScoreThreads>(srow, nb, a.K, a.s_pages, a.w_pages, keys,
-                              a.sel + ((size_t)b * a.Hkv + h) * a.K,
-                              a.sel_count + (size_t)b * a.Hkv + h,
-                              a.page_table + (size_t)b * a.max_pages,
-                              a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.K : nullptr);
+  for (int i = tot + tid; i < K; i += NT) {
+    out[i] = -1;
+    if (phys_out) phys_out[i] = -1;
+  }
+  if (tid == 0) *cnt_out = tot;
 }
 
-cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
-                                int n_tail, const int32_t* page_table, const int32_t* seq_lens,
-                                float* scores, uint32_t* arrivals, int K, int sink_pages,
-                                int window_pages, int32_t* sel, int32_t* sel_count,
-                                int32_t* sel_phys, int32_t* status, cudaStream_t stream) {
-  ScoreArgs a;
-  a.sel_phys = sel_phys;
-  a.q = static_cast<const uint16_t*>(q);
-  a.summ = static_cast<uint4*>(summ);
-  a.k_cache = static_cast<const uint4*>(k_cache);
-  a.page_table = page_table;
-  a.seq_lens = seq_lens;
-  a.scores = scores;
-  a.arrivals = arrivals;
-  a.sel = sel;
-  a.sel_count = sel_count;
-  a.status = status;
-  a.Hq = g.Hq;
-  a.Hkv = g.Hkv;
-  a.P = g.P;
-  a.max_pages = g.max_pages;
-  a.n_pool = g.n_pool;
-  a.K = K;
-  a.s_pages = sink_pages;
-  a.w_pages = window_pages;
-  a.n_tail = n_tail;
-  const int ntiles = (g.max_pages + kPagesPerCta - 1) / kPagesPerCta;
-  const size_t smem = (size_t)g.max_pages * sizeof(uint32_t);
-  void (*kern)(const ScoreArgs);
-  if (g.Dk == 64)
-    kern = score_select_kernel<64>;
-  else if (g.Dk == 128)
-    kern = score_select_kernel<128>;
-  else
-    return cudaErrorInvalidValue;
-  if (smem > 48 * 1024) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, void** args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ntiles * g.Hkv, g.B);
-  cfg.blockDim = dim3(kScoreThreads);
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -405,7 +653,111 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+// Tile shape of the scoring grid for geometry g (see ScoreArgs).
+static void score_shape(const sa_geom& g, ScoreArgs* a) {
+  const int D = g.Dk;
+  int hg = 1;  // power of two dividing Hkv, at most 2 KB of summaries per page slot
+  while (hg * 2 * 4 * D <= 2048 && g.Hkv % (hg * 2) == 0) hg *= 2;
+  a->HG = hg;
+  a->n_hg = g.Hkv / hg;
+  a->WPS = kScoreConsumers / hg;
+  a->NST = a->WPS <= 4 ? 4 : 8;  // a multiple of WPS: one warp group per stage slot
+  a->slot_bytes = hg * 4 * D + kSlotPad;
+  a->q_off = kTilePages * a->slot_bytes;
+  a->stage_bytes = (a->q_off + hg * (g.Hq / g.Hkv) * D * 2 + 127) & ~127;
+}
+
+static size_t score_smem(const sa_geom& g, const ScoreArgs& a) {
+  return 128 + (size_t)a.NST * a.stage_bytes + (size_t)(g.B + 1) * 4 +
+         (size_t)kMaxTilesPerCta * kTilePages * 4 + (size_t)5 * kMaxTilesPerCta * 4;
+}
+
+int score_ctas(const sa_geom& g, int sms) {
+  ScoreArgs a;
+  score_shape(g, &a);
+  const long long tiles = (long long)g.B * a.n_hg * ((g.max_pages + kTilePages - 1) / kTilePages);
+  const long long need = (tiles + kMaxTilesPerCta - 1) / kMaxTilesPerCta;
+  long long n = tiles < sms ? tiles : sms;
+  if (need > n) n = need;
+  return (int)(n > 0 ? n : 1);
+}
+
+bool score_supported(const sa_geom& g) {
+  if (!(g.Dk == 64 || g.Dk == 128)) return false;
+  ScoreArgs a;
+  score_shape(g, &a);
+  return score_smem(g, a) <= (size_t)kScoreSmemLimit;
+}
+
+cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
+                                int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+                                float* scores, int n_cta, int K, int sink_pages,
+                                int window_pages, int32_t* sel, int32_t* sel_count,
+                                int32_t* sel_phys, int32_t* status, cudaStream_t stream) {
+  ScoreArgs a;
+  a.q = static_cast<const uint16_t*>(q);
+  a.summ = static_cast<const uint8_t*>(summ);
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.scores = scores;
+  a.status = status;
+  a.B = g.B;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.G = g.Hq / g.Hkv;
+  a.P = g.P;
+  a.max_pages = g.max_pages;
+  a.n_pool = g.n_pool;
+  score_shape(g, &a);
+  const size_t smem = score_smem(g, a);
+  const void* kern;
+  const void* skern;
+  if (g.Dk == 64) {
+    kern = reinterpret_cast<const void*>(score_stream_kernel<64>);
+    skern = reinterpret_cast<const void*>(select_kernel<64>);
+  } else if (g.Dk == 128) {
+    kern = reinterpret_cast<const void*>(score_stream_kernel<128>);
+    skern = reinterpret_cast<const void*>(select_kernel<128>);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&a};
+  e = launch_pdl(kern, dim3(n_cta), dim3(kScoreThreads), smem, stream, args);
+  if (e != cudaSuccess) return e;
+
+  SelectArgs s;
+  s.q = a.q;
+  s.summ = static_cast<uint4*>(summ);
+  s.k_cache = n_tail > 0 ? static_cast<const uint4*>(k_cache) : nullptr;
+  s.page_table = page_table;
+  s.seq_lens = seq_lens;
+  s.scores = scores;
+  s.sel = sel;
+  s.sel_count = sel_count;
+  s.sel_phys = sel_phys;
+  s.status = status;
+  s.Hq = g.Hq;
+  s.Hkv = g.Hkv;
+  s.P = g.P;
+  s.max_pages = g.max_pages;
+  s.n_pool = g.n_pool;
+  s.K = K;
+  s.s_pages = sink_pages;
+  s.w_pages = window_pages;
+  s.n_tail = n_tail < kMaxTail ? n_tail : kMaxTail;
+  const size_t keys_bytes = (size_t)g.max_pages * 4;
+  s.ptab_in_smem = 2 * keys_bytes <= (size_t)200 * 1024;
+  const size_t ssmem = s.ptab_in_smem ? 2 * keys_bytes : keys_bytes;
+  e = cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+  if (e != cudaSuccess) return e;
+  void* sargs[] = {&s};
+  return launch_pdl(skern, dim3(g.Hkv, g.B), dim3(kSelectThreads), ssmem, stream, sargs);
 }
 
 }  // namespace sa

@@ -133,6 +133,33 @@ def test_decode_parity_small(kw):
     full_parity(case, res)
 
 
+@pytest.mark.parametrize("mode", ["zero_q", "quantized"])
+def test_selection_exact_ties_lowest_index(mode):
+    # Scores with many exact ties around the k-th place, computed exactly on both sides
+    # (all zero, or small integer sums): the lowest page indices must win, bit-exactly.
+    case = synth.decode_case("tiny", B=2, seq_lens=[4096, 3000], Hkv=2, Hq=8, budget=512,
+                             sink=16, window=64, seed=61)
+    rng = np.random.default_rng(61)
+    if mode == "zero_q":
+        case.q[...] = 0
+    else:
+        vals = np.array([0xBF80, 0x0000, 0x3F80], dtype=np.uint16)          # -1, 0, 1
+        case.q[...] = vals[rng.integers(0, 3, size=case.q.shape)]
+        kv = np.array([0xC000, 0xBF80, 0x0000, 0x3F80, 0x4000], dtype=np.uint16)  # -2..2
+        case.k_cache[...] = kv[rng.integers(0, 5, size=case.k_cache.shape)]
+    res = run_decode(DevCase(case))
+    g = case.geom
+    summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    sc = oracle.page_scores(g, case.q, summ, case.page_table, case.seq_lens)
+    o_sel, o_cnt = oracle.select_pages(g, sc, case.seq_lens, case.budget, case.sink,
+                                       case.window)
+    assert np.array_equal(res["cnt"], o_cnt)
+    assert np.array_equal(res["sel"], o_sel)
+    fin = np.isfinite(sc)
+    assert np.array_equal(res["scores"][fin], sc[fin].astype(np.float32))
+    full_parity(case, res)
+
+
 def test_budget_covers_all_pages_equals_dense():
     case = synth.decode_case("tiny", B=2, seq_lens=[1234, 4096], Hkv=2, Hq=8, budget=4096,
                              poison="nan")
