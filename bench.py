@@ -2,17 +2,19 @@
 
 One step = one decode step of a 32-layer model with Llama-3.1-8B attention geometry
 (batch 8, 32 query / 8 KV heads, head dim 128, 32768 tokens per sequence, page 16,
-token budget 2048 = sink 64 + window 512 + top-k): for every layer, sa_select_pages
-refreshes the summary of each sequence's newest page, scores every page and selects
-the top pages (one fused kernel), and sa_attend_selected runs split-KV attention over
-the gathered pages with the merge fused in (one persistent kernel) -- the two halves
-of sa_sparse_decode, called separately so the bench can time each.
-Every layer owns its own KV pool, so a step touches ~4.3 GB (> L2) and nothing is
-served from L2 across layers.
+token budget 2048 = sink 64 + window 512 + top-k).  Per layer, sa_select_pages scores
+every page against the query (streaming kernel) and selects the top pages (per-pair
+select kernel, which also refreshes the summary of each sequence's newest page), then
+sa_attend_selected runs split-KV attention over the gathered pages (attention kernel
+plus the merge kernel of the pairs split across warps) -- the two halves of
+sa_sparse_decode.  Every layer owns its own KV pool, so a step touches ~4.3 GB (> L2)
+and nothing is served from L2 across layers.
 
 Metric: sparse-decode seq*heads/s = (sequence, query head) attention outputs of one
-layer-call per second, whole job.  Also printed: achieved HBM GB/s of the whole step
-and, in "roofline", of the dominant kernel, against MEASURED_PEAKS.json.
+layer-call per second, whole job.  The headline is timed on a CUDA graph of the step
+with no event inside it; a second graph with an event between the two halves of every
+layer gives the per-phase times behind "roofline" (events between kernels cost the
+programmatic overlap of neighbouring kernels, so that pass is slightly slower).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama32k|llama128k|ragged]
   python bench.py --impl reference ...   (the CPU oracle on a bounded sample)
@@ -53,7 +55,6 @@ def parse():
     ap.add_argument("--layers", type=int, default=None,
                     help="layer pools per step (default 32 for llama32k, 8 otherwise)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--no-parity", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -271,15 +272,34 @@ def run_native(args, rank, world, dist):
     sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, P)
     step_bytes = L_layers * (sel_b + att_b + upd_b)
 
-    # capture one step (with per-layer events) in a CUDA graph
+    # the dominant kernel alone (page scoring of every layer), an event pair per launch
+    ev_sc = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+             for _ in range(L_layers)]
+    scores_buf = torch.empty((g.B, g.Hkv, g.max_pages), dtype=torch.float32, device=dev)
+
+    def score_only():
+        for l in range(L_layers):
+            ev_sc[l][0].record()
+            sa.page_scores(g, qs[l], summs[l], pt, sl, ws, scores=scores_buf)
+            ev_sc[l][1].record()
+
+    # capture: the step without events (headline), the step with per-phase events, and
+    # the scoring launches with per-launch events
     stream = torch.cuda.Stream()
     stream.wait_stream(torch.cuda.current_stream())
     graph = torch.cuda.CUDAGraph()
+    graph_ev = torch.cuda.CUDAGraph()
+    graph_sc = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         step(True)                      # warm the stream before capture
+        score_only()
         torch.cuda.synchronize()
         with torch.cuda.graph(graph, stream=stream):
+            step(False)
+        with torch.cuda.graph(graph_ev, stream=stream):
             step(True)
+        with torch.cuda.graph(graph_sc, stream=stream):
+            score_only()
     torch.cuda.synchronize()
 
     with torch.cuda.stream(stream):
@@ -293,8 +313,6 @@ def run_native(args, rank, world, dist):
     time.sleep(0.3)
     t0e = torch.cuda.Event(enable_timing=True)
     t1e = torch.cuda.Event(enable_timing=True)
-    sel_ms = np.zeros(L_layers)
-    att_ms = np.zeros(L_layers)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         t0e.record(stream)
@@ -303,10 +321,6 @@ def run_native(args, rank, world, dist):
         t1e.record(stream)
     torch.cuda.synchronize()
     total_ms = t0e.elapsed_time(t1e)
-    # per-phase durations: events of the last replay (identical work every replay)
-    for l in range(L_layers):
-        sel_ms[l] = ev[l][0].elapsed_time(ev[l][1])
-        att_ms[l] = ev[l][1].elapsed_time(ev[l][2])
     clk = clocks.stop()
     if dist is not None:
         import torch.distributed as tdist
@@ -317,6 +331,24 @@ def run_native(args, rank, world, dist):
     units_per_step = g.B * g.Hq * L_layers
     value = units_per_step * world / (ms_per_step * 1e-3)
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # ---- per-phase durations (events on the launching stream), averaged over replays
+    sel_ms = np.zeros(L_layers)
+    att_ms = np.zeros(L_layers)
+    n_ev = max(3, args.steps // 2)
+    sc_ms = np.zeros(L_layers)
+    with torch.cuda.stream(stream):
+        for _ in range(n_ev):
+            graph_ev.replay()
+            torch.cuda.synchronize()
+            for l in range(L_layers):
+                sel_ms[l] += ev[l][0].elapsed_time(ev[l][1]) / n_ev
+                att_ms[l] += ev[l][1].elapsed_time(ev[l][2]) / n_ev
+        for _ in range(n_ev):
+            graph_sc.replay()
+            torch.cuda.synchronize()
+            for l in range(L_layers):
+                sc_ms[l] += ev_sc[l][0].elapsed_time(ev_sc[l][1]) / n_ev
 
     # ---- e2e through the public API with host buffers: q H2D + out/lse D2H every step
     q_host = [torch.empty(qs[l].shape, dtype=torch.int16).pin_memory() for l in range(L_layers)]
@@ -346,27 +378,22 @@ def run_native(args, rank, world, dist):
         tt = torch.tensor([e2e_ms], device=dev)
         tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
         e2e_ms = float(tt.item())
+    assert ws.status() == sa.SA_OK
     h2d = sum(int(x.numel()) * 2 for x in q_host)
     d2h = sum(int(x.numel()) * 4 for x in o_host) + sum(int(x.numel()) * 4 for x in l_host)
-
-    # ---- sampled parity at full size: layer 0 against the oracle
-    parity = None
-    if rank == 0 and not args.no_parity:
-        parity = full_size_parity(case, outs[0], lses[0], sel, cnt, sa, g, ks, vs, qs, summs, pt,
-                                  sl, ws, dev)
 
     if rank != 0:
         return 0
     att_mean = float(att_ms.mean())
     sel_mean = float(sel_ms.mean())
-    dom_is_att = att_mean >= sel_mean
-    dom_ms = att_mean if dom_is_att else sel_mean
-    dom_bytes = att_b if dom_is_att else sel_b
+    sc_mean = float(sc_ms.mean())
+    # page scoring: summaries + page-table entries + queries of one layer per launch
+    dom_kernel, dom_bytes, dom_ms = "score_stream_kernel", sel_b, sc_mean
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     cpu_v, cpu_done, cpu_t = (None, 0, 0.0)
     if world == 1:
         cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds)
-    launches_per_layer = 2  # score+select (with the tail refresh), attention (+merge)
+    launches_per_layer = 4  # score, select (+ tail refresh), attention, merge
     line = {
         "metric": "sparse-decode seq*heads/s",
         "value": value,
@@ -390,15 +417,18 @@ def run_native(args, rank, world, dist):
             "parallelism": "replicas (batch split), no collective" if world > 1 else "1 GPU",
             "step_hbm_gbs": step_gbs,
             "step_frac_of_hbm_peak": step_gbs / hbm_peak,
-            "select_us_per_layer": sel_mean * 1e3,
-            "attend_us_per_layer": att_mean * 1e3,
+            "us_per_layer": ms_per_step * 1e3 / L_layers,
+            "select_pages_us_alone": sel_mean * 1e3,
+            "attend_selected_us_alone": att_mean * 1e3,
+            "page_scores_us_alone": sc_mean * 1e3,
             "algorithmic_bytes_per_layer": sel_b + att_b + upd_b,
         },
         "roofline": {
-            "kernel": "attend_gqa_kernel" if dom_is_att else "score_select_kernel",
+            "kernel": dom_kernel,
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "peak_kind": peak_kind + " (burst copy)",
-            "traffic": None,
+            "bytes_per_launch": dom_bytes,
+            "traffic": recorded_traffic(dom_kernel, args.workload),
         },
         "cpu_baseline": None if cpu_v is None else {
             "value": cpu_v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
@@ -408,40 +438,28 @@ def run_native(args, rank, world, dist):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_layer * L_layers * args.steps,
         "clocks": clk,
-        "parity": parity,
     }
     print(json.dumps(line, default=_json_default), flush=True)
     return 0
 
 
-def full_size_parity(case, out0, lse0, sel, cnt, sa, g, ks, vs, qs, summs, pt, sl, ws, dev):
-    """Layer 0 at full size, in the bench's launch configuration, against the oracle:
-    selection bit-exact (tie band aside) and attention within tolerance for every
-    sequence and head."""
-    import torch
-    import oracle
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from parity import check_attention, check_selection
-    sa.select_pages(g, qs[0], summs[0], pt, sl, case.budget, case.sink, case.window, ws,
-                    sel=sel, sel_count=cnt)
-    sa.attend_selected(g, qs[0], ks[0], vs[0], pt, sl, sel, cnt, case.scale, ws, out=out0,
-                       lse=lse0)
-    torch.cuda.synchronize()
-    gs, gc = sel.cpu().numpy(), cnt.cpu().numpy()
-    summ = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
-    gsumm = summs[0].cpu().numpy().view(np.uint16)
-    summ_ok = bool(np.array_equal(gsumm, summ))
-    sc = oracle.page_scores(case.geom, case.q, summ, case.page_table, case.seq_lens)
-    osel, ocnt = oracle.select_pages(case.geom, sc, case.seq_lens, case.budget, case.sink,
-                                     case.window)
-    tied = check_selection(case.geom, case.seq_lens, case.budget, case.sink, case.window, sc,
-                           osel, ocnt, gs, gc)
-    o, l = oracle.attend(case.geom, case.q, case.k_cache, case.v_cache, case.page_table,
-                         case.seq_lens, gs if tied else osel, ocnt, case.scale)
-    err, rel, lerr = check_attention(out0.cpu().numpy(), lse0.cpu().numpy(), o, l)
-    return {"layer": 0, "summaries_bit_exact": summ_ok, "selection_bit_exact": not tied,
-            "tie_band_units": len(tied), "out_max_abs": err, "out_rel_l2": rel,
-            "lse_max_abs": lerr, "outputs_checked": int(o.shape[0] * o.shape[1])}
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
+    there is none for this workload or the kernel's source changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("workload") != workload:
+        return None
+    src = os.path.join(ROOT, "paged_kv_cache_sa_b200", "csrc", rec["source"])
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return rec["dram_bytes_per_launch"] if sha == rec["source_sha256"] else None
 
 
 def main():

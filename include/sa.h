@@ -129,6 +129,21 @@ int sa_update_summaries(const sa_geom* g, const void* k_cache, const int32_t* pa
                         const int32_t* seq_lens, int n_tail_pages, void* summ, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * (2) Page scoring alone  [SE hook-point paragraph (Quest): the query-aware page
+ * bound].  scores[b][h][p] = max over the G query heads g of KV head h of
+ * sum_c max(q[b][h*G+g][c] * kmax_c, q[b][h*G+g][c] * kmin_c) for p < n_b, with
+ * (kmin, kmax) = summ[page_table[b][p]][h]; -inf for n_b <= p < max_pages.  fp32,
+ * summation order unspecified.  q: [B][Hq][Dk] bf16, 16-byte aligned; summ as written
+ * by sa_page_summaries; scores: [B][Hkv][max_pages] fp32, caller-owned.  ws: any
+ * workspace of at least 256 bytes (only its status word is used: page-table entries
+ * outside [0, n_pool) set SA_ERR_DEVICE_CHECK there and score as 0).  Asynchronous on
+ * `stream`; argument errors are returned before any launch.
+ * ------------------------------------------------------------------------------ */
+int sa_page_scores(const sa_geom* g, const void* q, const void* summ,
+                   const int32_t* page_table, const int32_t* seq_lens, float* scores, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * (2)+(3) Page scoring and top-k selection  [SE hook-point paragraph (Quest);
  * VX section 1 ("top pages"); SC Tri-shape section (sink + local window)].
  * K = budget/P pages per (sequence, KV head).  If n_b = ceil(seq_lens[b]/P) <= K

@@ -40,7 +40,8 @@ STATUS = {0: "SA_OK", -1: "SA_ERR_INVALID_ARG", -2: "SA_ERR_UNSUPPORTED", -3: "S
 # every symbol include/sa.h declares
 EXPORTS = ["sa_status_string", "sa_version", "sa_decode_workspace_size", "sa_prune_workspace_size",
            "sa_workspace_init", "sa_workspace_status", "sa_page_summaries", "sa_update_summaries",
-           "sa_select_pages", "sa_sparse_decode", "sa_attend_selected", "sa_prune_compact"]
+           "sa_page_scores", "sa_select_pages", "sa_sparse_decode", "sa_attend_selected",
+           "sa_prune_compact"]
 
 
 class SaError(RuntimeError):
@@ -91,6 +92,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sa_workspace_status": ([vp, vp], i32),
         "sa_page_summaries": ([G, vp, vp, vp, vp, vp], i32),
         "sa_update_summaries": ([G, vp, vp, vp, i32, vp, vp], i32),
+        "sa_page_scores": ([G, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "sa_select_pages": ([G, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, sz,
                              vp], i32),
         "sa_sparse_decode": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, vp,
@@ -178,6 +180,19 @@ def update_summaries(geom: Geometry, k_cache, page_table, seq_lens, summ, n_tail
                                    _ptr(seq_lens), int(n_tail_pages), _ptr(summ),
                                    _stream(stream)), "sa_update_summaries")
     return summ
+
+
+def page_scores(geom: Geometry, q, summ, page_table, seq_lens, ws: Workspace, scores=None,
+                stream=None):
+    """Page scores alone: [B][Hkv][max_pages] fp32 (-inf past each sequence's pages)."""
+    if scores is None:
+        scores = torch.empty((geom.B, geom.Hkv, geom.max_pages), dtype=torch.float32,
+                             device=q.device)
+    g = geom.c()
+    _check(lib.sa_page_scores(ctypes.byref(g), _ptr(q), _ptr(summ), _ptr(page_table),
+                              _ptr(seq_lens), _ptr(scores), _ptr(ws.buf), ws.nbytes,
+                              _stream(stream)), "sa_page_scores")
+    return scores
 
 
 def select_pages(geom: Geometry, q, summ, page_table, seq_lens, budget, sink, window,

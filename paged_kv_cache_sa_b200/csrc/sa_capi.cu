@@ -228,6 +228,21 @@ static int run_attend(const sa_geom& g, const DecodePlan& plan, uint8_t* w, cons
   return cuda_status(launch_attend(g, c, s));
 }
 
+SA_EXPORT int sa_page_scores(const sa_geom* g, const void* q, const void* summ,
+                             const int32_t* page_table, const int32_t* seq_lens, float* scores,
+                             void* ws, size_t ws_bytes, void* stream) {
+  int st = check_geom(g);
+  if (st != SA_OK) return st;
+  if (!q || !summ || !page_table || !seq_lens || !scores) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(summ)) return SA_ERR_INVALID_ARG;
+  if (!is_gqa(*g)) return SA_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < 256 || !aligned16(ws)) return SA_ERR_WORKSPACE;
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  return cuda_status(launch_score(*g, q, summ, page_table, seq_lens, scores,
+                                  score_ctas(*g, sm_count()), &hdr->status_bits,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
 SA_EXPORT int sa_select_pages(const sa_geom* g, const void* q, void* summ,
                               const int32_t* page_table, const int32_t* seq_lens, int budget,
                               int sink, int window, const void* k_cache, int n_tail_refresh,

@@ -31,6 +31,9 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
                                 int window_pages, int32_t* sel, int32_t* sel_count,
                                 int32_t* sel_phys, int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
+                         const int32_t* page_table, const int32_t* seq_lens, float* scores,
+                         int n_cta, int32_t* status, cudaStream_t stream);
 int score_ctas(const sa_geom& g, int sms);
 bool score_supported(const sa_geom& g);
 

@@ -283,6 +283,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
       if (lane == 0) mbar_arrive(&empty_bar[s]);
     }
   }
+  if (warp == kScoreConsumers) {
+    // scores past each sequence's last page are -inf (pairs spread over the CTAs)
+    for (int pr = c; pr < a.B * a.Hkv; pr += n_cta) {
+      const int b = pr / a.Hkv;
+      const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
+      float* srow = a.scores + (size_t)pr * a.max_pages;
+      for (int p = (L + a.P - 1) / a.P + lane; p < a.max_pages; p += 32) srow[p] = -INFINITY;
+    }
+  }
   __syncthreads();
   if (abort_flag && warp == kScoreConsumers && lane == 0) {
     // a wait expired: give copies still in flight a bounded time (10 ms) to land
@@ -453,7 +462,6 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
   int32_t* cnt_out = a.sel_count + (size_t)b * a.Hkv + h;
   int32_t* phys_out = a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.K : nullptr;
   for (int i = tid; i < n_tail; i += NT) srow[tail0 + i] = tail_score[i];
-  for (int p = nb + tid; p < a.max_pages; p += NT) srow[p] = -INFINITY;
   const int K = a.K;
   if (nb <= K) {  // everything fits the budget
     for (int i = tid; i < K; i += NT) {
@@ -692,11 +700,9 @@ bool score_supported(const sa_geom& g) {
   return score_smem(g, a) <= (size_t)kScoreSmemLimit;
 }
 
-cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
-                                int n_tail, const int32_t* page_table, const int32_t* seq_lens,
-                                float* scores, int n_cta, int K, int sink_pages,
-                                int window_pages, int32_t* sel, int32_t* sel_count,
-                                int32_t* sel_phys, int32_t* status, cudaStream_t stream) {
+static ScoreArgs make_score_args(const sa_geom& g, const void* q, const void* summ,
+                                 const int32_t* page_table, const int32_t* seq_lens,
+                                 float* scores, int32_t* status) {
   ScoreArgs a;
   a.q = static_cast<const uint16_t*>(q);
   a.summ = static_cast<const uint8_t*>(summ);
@@ -712,27 +718,45 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
   a.max_pages = g.max_pages;
   a.n_pool = g.n_pool;
   score_shape(g, &a);
+  return a;
+}
+
+cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
+                         const int32_t* page_table, const int32_t* seq_lens, float* scores,
+                         int n_cta, int32_t* status, cudaStream_t stream) {
+  ScoreArgs a = make_score_args(g, q, summ, page_table, seq_lens, scores, status);
   const size_t smem = score_smem(g, a);
   const void* kern;
-  const void* skern;
-  if (g.Dk == 64) {
+  if (g.Dk == 64)
     kern = reinterpret_cast<const void*>(score_stream_kernel<64>);
-    skern = reinterpret_cast<const void*>(select_kernel<64>);
-  } else if (g.Dk == 128) {
+  else if (g.Dk == 128)
     kern = reinterpret_cast<const void*>(score_stream_kernel<128>);
-    skern = reinterpret_cast<const void*>(select_kernel<128>);
-  } else {
+  else
     return cudaErrorInvalidValue;
-  }
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   void* args[] = {&a};
-  e = launch_pdl(kern, dim3(n_cta), dim3(kScoreThreads), smem, stream, args);
-  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(n_cta), dim3(kScoreThreads), smem, stream, args);
+}
 
+cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
+                                int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+                                float* scores, int n_cta, int K, int sink_pages,
+                                int window_pages, int32_t* sel, int32_t* sel_count,
+                                int32_t* sel_phys, int32_t* status, cudaStream_t stream) {
+  cudaError_t e =
+      launch_score(g, q, summ, page_table, seq_lens, scores, n_cta, status, stream);
+  if (e != cudaSuccess) return e;
+  const void* skern;
+  if (g.Dk == 64)
+    skern = reinterpret_cast<const void*>(select_kernel<64>);
+  else if (g.Dk == 128)
+    skern = reinterpret_cast<const void*>(select_kernel<128>);
+  else
+    return cudaErrorInvalidValue;
   SelectArgs s;
-  s.q = a.q;
+  s.q = static_cast<const uint16_t*>(q);
   s.summ = static_cast<uint4*>(summ);
   s.k_cache = n_tail > 0 ? static_cast<const uint4*>(k_cache) : nullptr;
   s.page_table = page_table;

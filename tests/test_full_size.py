@@ -1,0 +1,64 @@
+"""Parity at the full benchmark sizes, in the launch configuration bench.py times.
+
+Per layer, bench.py calls select_pages (newest page's summary refreshed, physical pages of
+the selection returned) and then attend_selected with those physical pages.  Here the same
+two calls run once on the full Llama-3.1-8B-geometry workloads (batch 8, 32/8 heads,
+head dim 128, 32K or 128K tokens per sequence) and every output is compared with the
+oracle: summaries bit-exact, selection bit-exact outside the tie band, attention within
+the stated tolerance.
+"""
+
+import numpy as np
+import pytest
+
+import synth
+import oracle
+from parity import DevCase, check_attention, check_selection, u16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("wl", ["llama32k", "llama128k"])
+def test_full_size_bench_launch_config(wl):
+    import torch
+    import paged_kv_cache_sa_b200 as sa
+    case = synth.decode_case(wl)
+    dc = DevCase(case)
+    g = dc.g
+    K = case.budget // g.P
+    sa.page_summaries(g, dc.k, dc.pt, dc.sl, dc.summ)
+    ws = sa.Workspace.for_decode(g, case.budget)
+    sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((g.B, g.Hkv), dtype=torch.int32, device="cuda")
+    phys = torch.empty_like(sel)
+    scores = torch.empty((g.B, g.Hkv, g.max_pages), dtype=torch.float32, device="cuda")
+    sa.select_pages(g, dc.q, dc.summ, dc.pt, dc.sl, case.budget, case.sink, case.window, ws,
+                    sel=sel, sel_count=cnt, k_cache=dc.k, n_tail_refresh=1, sel_phys=phys,
+                    scores=scores)
+    out, lse = sa.attend_selected(g, dc.q, dc.k, dc.v, dc.pt, dc.sl, sel, cnt, case.scale, ws,
+                                  sel_phys=phys)
+    assert ws.status() == sa.SA_OK
+    gs, gc = sel.cpu().numpy(), cnt.cpu().numpy()
+
+    summ = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    assert np.array_equal(u16(dc.summ), summ)
+    sc = oracle.page_scores(case.geom, case.q, summ, case.page_table, case.seq_lens)
+    fin = np.isfinite(sc)
+    gsc = scores.cpu().numpy()
+    assert np.array_equal(fin, np.isfinite(gsc))
+    assert np.allclose(gsc[fin], sc[fin], rtol=1e-5, atol=1e-4)
+    osel, ocnt = oracle.select_pages(case.geom, sc, case.seq_lens, case.budget, case.sink,
+                                     case.window)
+    tied = check_selection(case.geom, case.seq_lens, case.budget, case.sink, case.window, sc,
+                           osel, ocnt, gs, gc)
+    # the physical pages handed to attention are the page-table entries of the selection
+    pt = case.page_table
+    gp = phys.cpu().numpy()
+    for b in range(g.B):
+        for h in range(g.Hkv):
+            c = gc[b, h]
+            assert np.array_equal(gp[b, h, :c], pt[b, gs[b, h, :c]])
+            assert (gp[b, h, c:] == -1).all()
+    o, l = oracle.attend(case.geom, case.q, case.k_cache, case.v_cache, case.page_table,
+                         case.seq_lens, gs if tied else osel, ocnt, case.scale)
+    check_attention(out.cpu().numpy(), lse.cpu().numpy(), o, l)

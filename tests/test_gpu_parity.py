@@ -160,6 +160,29 @@ def test_selection_exact_ties_lowest_index(mode):
     full_parity(case, res)
 
 
+@pytest.mark.parametrize("kw", [dict(wl="tiny", B=3, seq_lens=[4096, 700, 0], Hkv=2, Hq=8),
+                                dict(wl="llama32k", B=2, L=(3000, 9000), seed=71),
+                                dict(wl="tiny", B=2, seq_lens=[5000, 33], Hkv=1, Hq=6, P=64,
+                                     budget=1024, sink=64, window=256)])
+def test_page_scores_alone(kw):
+    kw = dict(kw)
+    case = synth.decode_case(kw.pop("wl"), **kw)
+    dc = DevCase(case)
+    g = dc.g
+    sa.page_summaries(g, dc.k, dc.pt, dc.sl, dc.summ)
+    ws = sa.Workspace.for_decode(g, case.budget)
+    sc = torch.full((g.B, g.Hkv, g.max_pages), 7.0, dtype=torch.float32, device="cuda")
+    sa.page_scores(g, dc.q, dc.summ, dc.pt, dc.sl, ws, scores=sc)
+    assert ws.status() == sa.SA_OK
+    summ = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    ref = oracle.page_scores(case.geom, case.q, summ, case.page_table, case.seq_lens)
+    got = sc.cpu().numpy()
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(got))
+    assert np.isneginf(got[~fin]).all()
+    assert np.allclose(got[fin], ref[fin], rtol=1e-5, atol=1e-4)
+
+
 def test_budget_covers_all_pages_equals_dense():
     case = synth.decode_case("tiny", B=2, seq_lens=[1234, 4096], Hkv=2, Hq=8, budget=4096,
                              poison="nan")
