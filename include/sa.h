@@ -181,6 +181,35 @@ int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache, const
                      float* lse, int32_t* sel_out, int32_t* sel_count_out, void* ws,
                      size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------
+ * Allocation-free sparse decode.  The pages have no counterpart to this call: it is an
+ * engineering variant of sa_sparse_decode for callers that cannot hand the library a
+ * workspace.  Arguments, results and argument errors are those of sa_sparse_decode
+ * without (ws, ws_bytes); the workspace is instead a scratch array inside the library,
+ * a static device variable of SA_STATIC_SCRATCH_BYTES bytes per device, so nothing is
+ * allocated at run time (no cudaMalloc, no allocating library routine).
+ *  - Limit: a geometry and budget whose sa_decode_workspace_size exceeds
+ *    SA_STATIC_SCRATCH_BYTES is rejected with SA_ERR_WORKSPACE before any launch
+ *    (Llama-3.1-8B geometry, batch 8, 128K tokens, budget 2048 needs about 8 MB).
+ *  - Setup: the first call on a device, with that device current, looks the scratch up
+ *    with cudaGetSymbolAddress and zeroes its status word synchronously; make that
+ *    first call before any stream capture.
+ *  - Zeroing: only the scratch's status word must start at zero; every call clears it
+ *    again on `stream` after its kernels.
+ *  - status_out (nullable, device int32): receives, on `stream`, the bit-OR of the
+ *    device-detected errors of this call ((1 << -status) per error, 0 when none).
+ *  - Concurrency: the scratch is shared by all calls on a device.  Calls that can
+ *    overlap in time (other streams, other host threads) race on it; the caller must
+ *    serialise them.
+ * ------------------------------------------------------------------------------ */
+#define SA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+int sa_sparse_decode_noalloc(const sa_geom* g, const void* q, const void* k_cache,
+                             const void* v_cache, void* summ, const int32_t* page_table,
+                             const int32_t* seq_lens, int budget, int sink, int window,
+                             int n_tail_refresh, float scale, float* out, float* lse,
+                             int32_t* sel_out, int32_t* sel_count_out, int32_t* status_out,
+                             void* stream);
+
 /* Attention over a given selection (sel [B][Hkv][sel_stride], ascending logical
  * pages, sel_count [B][Hkv] <= sel_stride): the reuse of one layer's selected
  * indices at later layers [SE hook-point paragraph, OmniKV/DeltaKV].  `budget` for

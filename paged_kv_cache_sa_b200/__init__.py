@@ -33,6 +33,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libsa.so")
 
 SA_OK = 0
+SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE = -1, -2, -3
 STATUS = {0: "SA_OK", -1: "SA_ERR_INVALID_ARG", -2: "SA_ERR_UNSUPPORTED", -3: "SA_ERR_WORKSPACE",
           -4: "SA_ERR_CUDA", -5: "SA_ERR_DEVICE_CHECK", -6: "SA_ERR_TIMEOUT",
           -7: "SA_ERR_NO_SPACE"}
@@ -41,7 +42,7 @@ STATUS = {0: "SA_OK", -1: "SA_ERR_INVALID_ARG", -2: "SA_ERR_UNSUPPORTED", -3: "S
 EXPORTS = ["sa_status_string", "sa_version", "sa_decode_workspace_size", "sa_prune_workspace_size",
            "sa_workspace_init", "sa_workspace_status", "sa_page_summaries", "sa_update_summaries",
            "sa_page_scores", "sa_select_pages", "sa_sparse_decode", "sa_attend_selected",
-           "sa_prune_compact"]
+           "sa_prune_compact", "sa_sparse_decode_noalloc"]
 
 
 class SaError(RuntimeError):
@@ -97,6 +98,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                              vp], i32),
         "sa_sparse_decode": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, vp,
                               vp, vp, vp, vp, sz, vp], i32),
+        "sa_sparse_decode_noalloc": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                      ctypes.c_float, vp, vp, vp, vp, vp, vp], i32),
         "sa_attend_selected": ([G, vp, vp, vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp,
                                 vp, sz, vp], i32),
         "sa_prune_compact": ([G, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, sz,
@@ -231,6 +234,26 @@ def sparse_decode(geom: Geometry, q, k_cache, v_cache, summ, page_table, seq_len
                                 int(window), int(n_tail_refresh), float(scale), _ptr(out),
                                 _ptr(lse), _ptr(sel_out), _ptr(sel_count_out), _ptr(ws.buf),
                                 ws.nbytes, _stream(stream)), "sa_sparse_decode")
+    return out, lse
+
+
+def sparse_decode_noalloc(geom: Geometry, q, k_cache, v_cache, summ, page_table, seq_lens,
+                          budget, sink, window, scale, out=None, lse=None, sel_out=None,
+                          sel_count_out=None, status_out=None, n_tail_refresh: int = 0,
+                          stream=None):
+    """sa_sparse_decode on the library's static scratch (no workspace argument)."""
+    dev = q.device
+    if out is None:
+        out = torch.empty((geom.B, geom.Hq, geom.Dv), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((geom.B, geom.Hq), dtype=torch.float32, device=dev)
+    g = geom.c()
+    _check(lib.sa_sparse_decode_noalloc(ctypes.byref(g), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(summ), _ptr(page_table), _ptr(seq_lens), int(budget),
+                                        int(sink), int(window), int(n_tail_refresh), float(scale),
+                                        _ptr(out), _ptr(lse), _ptr(sel_out), _ptr(sel_count_out),
+                                        _ptr(status_out), _stream(stream)),
+           "sa_sparse_decode_noalloc")
     return out, lse
 
 

@@ -323,6 +323,56 @@ SA_EXPORT int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_ca
   return run_attend(*g, plan, w, q, k_cache, vc, page_table, seq_lens, sel, cnt,
                     reinterpret_cast<int32_t*>(w + plan.off_phys), plan.K, scale, out, lse, s);
 }
+namespace sa {
+// Scratch of sa_sparse_decode_noalloc: a static device variable, one per device.
+static __device__ __align__(256) uint8_t g_static_scratch[SA_STATIC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+static void* g_scratch_addr[kMaxDevices];
+static std::mutex g_scratch_mu;
+
+// Device address of the current device's scratch; looked up (and its status word
+// zeroed) on the first call for that device.
+static int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return SA_ERR_CUDA;
+    if (cudaMemset(p, 0, sizeof(WsHeader)) != cudaSuccess) return SA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return SA_OK;
+}
+}  // namespace sa
+
+SA_EXPORT int sa_sparse_decode_noalloc(const sa_geom* g, const void* q, const void* k_cache,
+                                       const void* v_cache, void* summ,
+                                       const int32_t* page_table, const int32_t* seq_lens,
+                                       int budget, int sink, int window, int n_tail_refresh,
+                                       float scale, float* out, float* lse, int32_t* sel_out,
+                                       int32_t* sel_count_out, int32_t* status_out,
+                                       void* stream) {
+  int st = check_geom(g);
+  if (st != SA_OK) return st;
+  if ((st = check_budget(*g, budget, sink, window)) != SA_OK) return st;
+  if (sa_decode_workspace_size(g, budget) > SA_STATIC_SCRATCH_BYTES) return SA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != SA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = sa_sparse_decode(g, q, k_cache, v_cache, summ, page_table, seq_lens, budget, sink, window,
+                        n_tail_refresh, scale, out, lse, sel_out, sel_count_out, scratch,
+                        SA_STATIC_SCRATCH_BYTES, stream);
+  if (st != SA_OK) return st;
+  if (status_out &&
+      cudaMemcpyAsync(status_out, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
+          cudaSuccess)
+    return SA_ERR_CUDA;
+  return cuda_status(cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s));
+}
+
 SA_EXPORT int sa_prune_compact(const sa_geom* g, const void* k_cache, const void* v_cache,
                                const int32_t* page_table, const int32_t* seq_lens,
                                const uint8_t* keep, const int32_t* free_pages, int64_t n_free,

@@ -19,7 +19,12 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def libpath():
-    from paged_kv_cache_sa_b200 import build as b
+    # build.py by path: importing the package first would load a possibly stale library
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_sa_build", os.path.join(ROOT, "paged_kv_cache_sa_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
     return b.build()
 
 
