@@ -294,7 +294,11 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     }
   } else {
     // ===================== consumer warps =====================
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // The producer alone waits for the previous grid (the wait makes its memory visible
+    // to this whole grid); consumers block on the hardware barrier until the tables,
+    // built after that wait, are ready.  (Every thread takes part in the early launch of
+    // the merge grid.)
+    asm volatile("griddepcontrol.launch_dependents;");
     named_bar(1, kThreads);  // tables ready
     const int r = lane >> 2, t = lane & 3;
     const uint32_t stage0 = smem_u32(stages);
@@ -486,8 +490,10 @@ struct MergeArgs {
 template <int D>
 __global__ void __launch_bounds__(128) attend_merge_kernel(const MergeArgs a) {
   constexpr int HS = D + 4;
-  constexpr int CH = 8;  // states in flight per lane
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int CH = 16;  // states in flight per lane
+  // one thread waits for the attention grid; the rest block on the CTA barrier
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+  __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;");
   const int lane = threadIdx.x & 31;
   const int wi = blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -582,6 +588,13 @@ static cudaError_t launch_attend_t(const sa_geom& g, const void* k_cache, const 
   if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(attend_gqa_kernel<D, P, NC, SPW>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // largest carveout for every decode kernel: neighbours can share an SM
+    e = cudaFuncSetAttribute(attend_gqa_kernel<D, P, NC, SPW>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attend_merge_kernel<D>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     configured = smem;
   }

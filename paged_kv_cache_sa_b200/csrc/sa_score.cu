@@ -83,7 +83,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
   uint8_t* stages = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   int* pre = reinterpret_cast<int*>(stages + (size_t)a.NST * a.stage_bytes);  // [B + 1]
-  int* ptab = pre + a.B + 1;                       // [kMaxTilesPerCta * 16]
+  int* nbs = pre + a.B + 1;                        // [B] pages per sequence
+  int* ptab = nbs + a.B;                           // [kMaxTilesPerCta * 16]
   int* t_b = ptab + kMaxTilesPerCta * kTilePages;  // per tile of the slice
   int* t_hg = t_b + kMaxTilesPerCta;
   int* t_p0 = t_hg + kMaxTilesPerCta;
@@ -103,9 +104,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
     abort_flag = 0;
     fence_mbar_init();
   }
+  // everything read below may come from the previous kernel of the stream: one thread
+  // waits for it (which makes its memory visible to this grid), the rest block on the
+  // CTA barrier
+  if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
-  // everything read below may come from the previous kernel of the stream
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
 
   if (warp == kScoreConsumers) {
@@ -119,6 +122,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
         const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
         const int nb = (L + a.P - 1) / a.P;
         n = a.n_hg * ((nb + kTilePages - 1) / kTilePages);
+        nbs[b] = nb;
       }
       int incl = n;
 #pragma unroll
@@ -141,8 +145,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
       const int b = find_seq(pre, a.B, u);
       const int ntb = (pre[b + 1] - pre[b]) / a.n_hg;  // tiles per head group
       const int rem = u - pre[b];
-      const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
-      const int nb = (L + a.P - 1) / a.P;
+      const int nb = nbs[b];
       t_b[i] = b;
       t_hg[i] = rem / ntb;
       t_p0[i] = (rem % ntb) * kTilePages;
@@ -454,10 +457,10 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
                                      G, ph, h, a.Hkv, a.P, min(a.P, L - lp * a.P), lane);
     if (lane == 0) tail_score[i] = sc;
   }
-  // 2. wait for the scores
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
+  // 2. wait for the scores (one thread; the rest block on the CTA barrier)
+  if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;");
   int32_t* out = a.sel + ((size_t)b * a.Hkv + h) * a.K;
   int32_t* cnt_out = a.sel_count + (size_t)b * a.Hkv + h;
   int32_t* phys_out = a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.K : nullptr;
@@ -623,24 +626,40 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
     }
   }
 
-  // 5. ascending list: forced pages and taken candidates
-  const int seg = (nb + NT - 1) / NT;
-  const int beg = min(nb, tid * seg), end = min(nb, beg + seg);
+  // 5. ascending list: forced pages and taken candidates.  Each warp owns a contiguous
+  // run of pages (a multiple of 32) and compacts it with ballots; one block barrier
+  // gives every warp its offset.
   auto taken = [&](int p) {
     if (p < a.s_pages || p >= wbeg) return true;
     const uint32_t key = keys[p];
     return key == kWin || (uint64_t)key >= thr;
   };
+  const int per_warp = ((nb + NT - 1) / NT) * 32;
+  const int w0 = min(nb, warp * per_warp), w1 = min(nb, w0 + per_warp);
   int n_sel = 0;
-  for (int p = beg; p < end; ++p) n_sel += taken(p);
-  int tot;
-  int pos = block_excl_scan<NT>(n_sel, warp_tot, &tot);
-  for (int p = beg; p < end; ++p) {
-    if (taken(p)) {
-      out[pos] = p;
-      if (phys_out) phys_out[pos] = ptab_s ? ptab_s[p] : ptab_g[p];
-      ++pos;
+  for (int p0 = w0; p0 < w1; p0 += 32) {
+    const int p = p0 + lane;
+    n_sel += __popc(__ballot_sync(0xffffffffu, p < w1 && taken(p)));
+  }
+  if (lane == 0) warp_tot[warp] = n_sel;
+  __syncthreads();
+  int pos = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const int v = warp_tot[w];
+    pos += w < warp ? v : 0;
+    tot += v;
+  }
+  for (int p0 = w0; p0 < w1; p0 += 32) {
+    const int p = p0 + lane;
+    const bool tk = p < w1 && taken(p);
+    const unsigned m = __ballot_sync(0xffffffffu, tk);
+    if (tk) {
+      const int at = pos + __popc(m & ((1u << lane) - 1u));
+      out[at] = p;
+      if (phys_out) phys_out[at] = ptab_s ? ptab_s[p] : ptab_g[p];
     }
+    pos += __popc(m);
   }
   for (int i = tot + tid; i < K; i += NT) {
     out[i] = -1;
@@ -679,7 +698,7 @@ static void score_shape(const sa_geom& g, ScoreArgs* a) {
 }
 
 static size_t score_smem(const sa_geom& g, const ScoreArgs& a) {
-  return 128 + (size_t)a.NST * a.stage_bytes + (size_t)(g.B + 1) * 4 +
+  return 128 + (size_t)a.NST * a.stage_bytes + (size_t)(2 * g.B + 1) * 4 +
          (size_t)kMaxTilesPerCta * kTilePages * 4 + (size_t)5 * kMaxTilesPerCta * 4;
 }
 
@@ -736,6 +755,10 @@ cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // every decode kernel prefers the largest shared-memory carveout, so that the next
+  // kernel's CTAs can become resident next to this one's (programmatic launch)
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
   void* args[] = {&a};
   return launch_pdl(kern, dim3(n_cta), dim3(kScoreThreads), smem, stream, args);
 }
@@ -779,6 +802,8 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
   s.ptab_in_smem = 2 * keys_bytes <= (size_t)200 * 1024;
   const size_t ssmem = s.ptab_in_smem ? 2 * keys_bytes : keys_bytes;
   e = cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(skern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   void* sargs[] = {&s};
   return launch_pdl(skern, dim3(g.Hkv, g.B), dim3(kSelectThreads), ssmem, stream, sargs);
