@@ -74,7 +74,10 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   p.off_pre = off;
   off += up256(((size_t)g.B * g.Hkv + 1) * 4);
   p.off_part = off;
-  off += up256(attend_partial_floats(g, p.n_cta) * 4);
+  // the latent geometry has no attention path here: no split states
+  if (!is_latent(g)) off += up256(attend_partial_floats(g, p.n_cta) * 4);
+  p.off_qs = off;  // latent geometry: sign-split query rows for the tensor-core scoring
+  if (is_latent(g)) off += up256(mla_qsplit_bytes(g));
   p.total = off;
   *plan = p;
   return true;
@@ -193,8 +196,21 @@ static int run_select(const sa_geom& g, const DecodePlan& plan, uint8_t* w, cons
                       void* summ, const void* k_cache, int n_tail, const int32_t* page_table,
                       const int32_t* seq_lens, int sink, int window, int32_t* sel, int32_t* cnt,
                       int32_t* phys, float* scores, cudaStream_t s) {
-  if (!is_gqa(g)) return SA_ERR_UNSUPPORTED;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
+  if (is_latent(g)) {
+    // newest pages' summaries first, then tensor-core scoring, then the selection
+    if (n_tail > 0) {
+      const int st = cuda_status(launch_summaries(g, k_cache, page_table, seq_lens, summ, n_tail, s));
+      if (st != SA_OK) return st;
+    }
+    int st = cuda_status(launch_score_mla(g, q, summ, w + plan.off_qs, page_table, seq_lens,
+                                          scores, &hdr->status_bits, s));
+    if (st != SA_OK) return st;
+    return cuda_status(launch_select(g, q, summ, nullptr, 0, page_table, seq_lens, scores, plan.K,
+                                     sink / g.P, window / g.P, sel, cnt, phys, &hdr->status_bits,
+                                     s));
+  }
+  if (!is_gqa(g)) return SA_ERR_UNSUPPORTED;
   return cuda_status(launch_score_select(
       g, q, summ, n_tail > 0 ? k_cache : nullptr, n_tail, page_table, seq_lens, scores,
       plan.n_score_cta, plan.K, sink / g.P, window / g.P, sel,
@@ -235,6 +251,13 @@ SA_EXPORT int sa_page_scores(const sa_geom* g, const void* q, const void* summ,
   if (st != SA_OK) return st;
   if (!q || !summ || !page_table || !seq_lens || !scores) return SA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(summ)) return SA_ERR_INVALID_ARG;
+  if (is_latent(*g)) {
+    if (!ws || ws_bytes < 256 + mla_qsplit_bytes(*g) || !aligned16(ws)) return SA_ERR_WORKSPACE;
+    WsHeader* hdr = static_cast<WsHeader*>(ws);
+    return cuda_status(launch_score_mla(*g, q, summ, static_cast<uint8_t*>(ws) + 256, page_table,
+                                        seq_lens, scores, &hdr->status_bits,
+                                        static_cast<cudaStream_t>(stream)));
+  }
   if (!is_gqa(*g)) return SA_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < 256 || !aligned16(ws)) return SA_ERR_WORKSPACE;
   WsHeader* hdr = static_cast<WsHeader*>(ws);
@@ -257,7 +280,7 @@ SA_EXPORT int sa_select_pages(const sa_geom* g, const void* q, void* summ,
   if (!aligned16(q) || !aligned16(summ) || (k_cache && !aligned16(k_cache)))
     return SA_ERR_INVALID_ARG;
   if ((size_t)g->max_pages * 4 > 200 * 1024) return SA_ERR_UNSUPPORTED;
-  if (!is_gqa(*g)) return SA_ERR_UNSUPPORTED;
+  if (!is_gqa(*g) && !is_latent(*g)) return SA_ERR_UNSUPPORTED;
   DecodePlan plan;
   make_decode_plan(*g, budget, &plan);
   if (!ws || ws_bytes < plan.total || !aligned16(ws)) return SA_ERR_WORKSPACE;

@@ -15,7 +15,7 @@ struct DecodePlan {
   int G;      // query heads per KV head
   int n_cta;        // attention CTAs (one per SM, more for very large selections)
   int n_score_cta;  // scoring CTAs (one per SM, more for very long sequences)
-  size_t off_scores, off_sel, off_cnt, off_phys, off_pre, off_part, total;
+  size_t off_scores, off_sel, off_cnt, off_phys, off_pre, off_part, off_qs, total;
 };
 
 bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan);
@@ -34,6 +34,19 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
 cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
                          const int32_t* page_table, const int32_t* seq_lens, float* scores,
                          int n_cta, int32_t* status, cudaStream_t stream);
+cudaError_t launch_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
+                          int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+                          float* scores, int K, int sink_pages, int window_pages, int32_t* sel,
+                          int32_t* sel_count, int32_t* sel_phys, int32_t* status,
+                          cudaStream_t stream);
+
+// Latent (MLA) geometry: sign-split queries (workspace, mla_qsplit_bytes) then scoring on
+// the tcgen05 tensor cores.
+size_t mla_qsplit_bytes(const sa_geom& g);
+cudaError_t launch_score_mla(const sa_geom& g, const void* q, const void* summ, void* qs,
+                             const int32_t* page_table, const int32_t* seq_lens, float* scores,
+                             int32_t* status, cudaStream_t stream);
+
 int score_ctas(const sa_geom& g, int sms);
 bool score_supported(const sa_geom& g);
 

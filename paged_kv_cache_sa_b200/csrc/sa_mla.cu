@@ -1,0 +1,346 @@
+// sa_mla.cu -- page scoring for the latent (MLA) geometry on the 5th-generation tensor
+// cores: 128 query heads share one 576-wide latent key per token.
+//
+// Method (the page bound of the SparseEngine blog's hook-point paragraph, Quest):
+//   S(b,p) = max over the 128 heads g of sum_c max(q_gc * kmax_c, q_gc * kmin_c)
+//          = max_g ( [kmin | kmax](p) . [min(q_g,0) | max(q_g,0)] ),
+// a dense contraction of length 2*576 = 1152 per (page, head), exactly (kmax >= kmin).
+//
+// Kernel shape.  One CTA per (sequence, tile of 128 logical pages).  D[page][head] =
+// A . B^T with A = the tile's summary rows (M = 128, gathered through the page table)
+// and B = the sequence's sign-split query rows (N = 128 heads), K = 1152 in 18 chunks of
+// 64.  Four producer warps stage each chunk with 16-byte cp.async copies into the
+// 128-byte-swizzled K-major layout the tensor core reads (8-row groups 1024 bytes
+// apart); one thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, 128x128x16)
+// into a 128-column TMEM accumulator and tcgen05.commit frees each stage; four
+// epilogue warps read their 32 TMEM lanes (one page row each) with tcgen05.ld and take
+// the max over the 128 head columns.  HBM-bound: 2 * 576 * 2 bytes per page.
+#include "sa_common.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+
+namespace mla {
+
+constexpr int kD = 576;            // latent key width
+constexpr int kG = 128;            // query heads
+constexpr int kK = 2 * kD;         // contraction length
+constexpr int kTile = 128;         // pages per CTA (UMMA M)
+constexpr int kChunk = 64;         // K elements per stage (128 bytes per row)
+constexpr int kChunks = kK / kChunk;  // 18
+constexpr int kStages = 4;
+constexpr int kRowBytes = kChunk * 2;               // 128
+constexpr int kOpBytes = kTile * kRowBytes;         // 16 KB per operand per stage
+constexpr int kStageBytes = 2 * kOpBytes;           // A | B
+constexpr int kThreads = 256;                       // 4 producer + 4 MMA/epilogue warps
+constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes;
+static_assert(kD % kChunk == 0, "a chunk never straddles the kmin/kmax halves");
+
+// ---- tcgen05 / cp.async wrappers ------------------------------------------------------
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major operand, 128-byte swizzle: rows 128 bytes apart, 8-row groups 1024 bytes
+// apart (stride-byte offset), descriptor version 1, layout type 2.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);  // start address
+  d |= (uint64_t)1 << 16;                         // leading-byte offset (unused here)
+  d |= (uint64_t)(1024 >> 4) << 32;               // stride-byte offset
+  d |= (uint64_t)1 << 46;                         // descriptor version
+  d |= (uint64_t)2 << 61;                         // 128-byte swizzle
+  return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace mla
+
+// Sign-split query rows of the latent geometry: qs[b][g] = [min(q,0) | max(q,0)] (bf16;
+// the half that does not apply is +0).  One thread per 8 channels.
+__global__ void __launch_bounds__(256) mla_qsplit_kernel(const uint4* __restrict__ q,
+                                                         uint4* __restrict__ qs, int rows) {
+  constexpr int CPR = mla::kD / 8;  // 72 chunks per query row
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  // the previous kernel of the stream may still read qs
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (i >= rows * CPR) return;
+  const int r = i / CPR, c = i % CPR;
+  const uint4 v = q[(size_t)r * CPR + c];
+  uint32_t w[4] = {v.x, v.y, v.z, v.w}, lo[4], hi[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t neg = ((w[e] >> 15) & 0x00010001u) * 0xFFFFu;  // negative halves
+    lo[e] = w[e] & neg;
+    hi[e] = w[e] & ~neg;
+  }
+  qs[(size_t)r * 2 * CPR + c] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  qs[(size_t)r * 2 * CPR + CPR + c] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+}
+
+struct MlaScoreArgs {
+  const uint8_t* summ;  // [n_pool][1][2][576] bf16
+  const uint8_t* qs;    // [B][128][1152] bf16, sign-split query rows
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  float* scores;  // [B][1][max_pages]
+  int32_t* status;
+  int P, max_pages, n_pool;
+};
+
+__global__ void __launch_bounds__(mla::kThreads, 1) score_mla_kernel(const MlaScoreArgs a) {
+  using namespace mla;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stages = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = blockIdx.x, b = blockIdx.y;
+  const int p0 = tile * kTile;
+
+  if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
+  const int nb = (L + a.P - 1) / a.P;
+  float* srow = a.scores + (size_t)b * a.max_pages;
+  if (p0 >= nb) {  // past the sequence: -inf scores, no tensor-core work
+    for (int p = p0 + tid; p < min(a.max_pages, p0 + kTile); p += kThreads) srow[p] = -INFINITY;
+    return;
+  }
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 128);  // the 128 producer threads
+      mbar_init(&empty_bar[s], 1);   // one tcgen05.commit
+    }
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {  // TMEM: 128 fp32 columns (one per head), 128 lanes (one per page)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base)),
+                 "r"(128)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  mla::tc_fence_before();
+  __syncthreads();
+  mla::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t st0 = smem_u32(stages);
+
+  if (warp < 4) {
+    // ===================== producers: 16-byte copies into swizzled stages ==========
+    // thread r owns row r of both operands: page p0 + r of A, head r of B
+    const int r = tid;
+    const int p = p0 + r;
+    int ph = -1;
+    if (p < nb) {
+      ph = a.page_table[(size_t)b * a.max_pages + p];
+      if (ph < 0 || ph >= a.n_pool) {
+        report(a.status, SA_ERR_DEVICE_CHECK);
+        ph = -1;
+      }
+    }
+    const uint8_t* arow = a.summ + (size_t)(ph < 0 ? 0 : ph) * (kK * 2);
+    const uint32_t asrc_bytes = ph < 0 ? 0u : 16u;  // zero-fill rows outside the sequence
+    const uint8_t* brow = a.qs + ((size_t)b * kG + r) * (kK * 2);
+    const uint32_t swz = (uint32_t)(r & 7);
+    for (int kc = 0; kc < kChunks; ++kc) {
+      const int s = kc % kStages;
+      if (kc >= kStages) {
+        bool ok = !*(volatile int*)&abort_flag;
+        if (ok && !mbar_wait(&empty_bar[s], ((kc / kStages) - 1) & 1)) {
+          report(a.status, SA_ERR_TIMEOUT);
+          atomicExch(&abort_flag, 1);
+        }
+      }
+      const uint32_t sa_ = st0 + s * kStageBytes + r * kRowBytes;
+      const uint32_t sb_ = sa_ + kOpBytes;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t off = (uint32_t)((u ^ swz) << 4);
+        cp_async16(sa_ + off, arow + kc * kRowBytes + u * 16, asrc_bytes);
+        cp_async16(sb_ + off, brow + kc * kRowBytes + u * 16, 16u);
+      }
+      cp_async_commit();
+      // the stage issued kStages-1 chunks ago has landed: publish it to the MMA thread
+      if (kc >= kStages - 1) {
+        cp_async_wait<kStages - 1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&full_bar[(kc - (kStages - 1)) % kStages]);
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    for (int kc = kChunks - (kStages - 1); kc < kChunks; ++kc) mbar_arrive(&full_bar[kc % kStages]);
+  } else {
+    // ===================== MMA issue (one thread) =====================
+    if (warp == 4 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kTile, kG);
+      bool ok = true;
+      for (int kc = 0; kc < kChunks && ok; ++kc) {
+        const int s = kc % kStages;
+        if (*(volatile int*)&abort_flag || !mbar_wait(&full_bar[s], (kc / kStages) & 1)) {
+          report(a.status, SA_ERR_TIMEOUT);
+          atomicExch(&abort_flag, 1);
+          ok = false;
+          break;
+        }
+        mla::tc_fence_after();
+        const uint32_t sa_ = st0 + s * kStageBytes;
+#pragma unroll
+        for (int k = 0; k < kChunk / 16; ++k) {
+          // advancing K by 16 elements = 32 bytes inside the swizzled 128-byte rows
+          umma_bf16(tmem, desc_sw128(sa_ + k * 32), desc_sw128(sa_ + kOpBytes + k * 32), idesc,
+                    (kc | k) != 0);
+        }
+        umma_commit(&empty_bar[s]);  // the stage is free once these MMAs have read it
+      }
+      umma_commit(&done_bar);  // all issued MMAs complete -> accumulator ready
+    }
+    __syncwarp();
+    // ===================== epilogue: lane (page) row max over 128 heads ==========
+    const int wq = warp - 4;  // TMEM lanes 32*wq .. 32*wq + 31
+    // warp-uniform: tcgen05.ld below is a .sync.aligned warp instruction
+    const bool ready = __all_sync(0xffffffffu, mbar_wait(&done_bar, 0));
+    mla::tc_fence_after();
+    float m = -INFINITY;
+    if (ready) {
+#pragma unroll
+      for (int c0 = 0; c0 < kG; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * wq) << 16) + c0, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i]);
+      }
+    } else if (lane == 0) {
+      report(a.status, SA_ERR_TIMEOUT);
+    }
+    const int p = p0 + 32 * wq + lane;
+    if (p < a.max_pages) srow[p] = (p < nb && !*(volatile int*)&abort_flag) ? m : -INFINITY;
+  }
+  mla::tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    mla::tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128)
+                 : "memory");
+  }
+}
+
+static cudaError_t launch_pdl_mla(const void* fn, dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+size_t mla_qsplit_bytes(const sa_geom& g) { return (size_t)g.B * mla::kG * mla::kK * 2; }
+
+cudaError_t launch_score_mla(const sa_geom& g, const void* q, const void* summ, void* qs,
+                             const int32_t* page_table, const int32_t* seq_lens, float* scores,
+                             int32_t* status, cudaStream_t stream) {
+  const int rows = g.B * mla::kG;
+  const int n_thr = rows * (mla::kD / 8);
+  const uint4* qv = static_cast<const uint4*>(q);
+  uint4* qsv = static_cast<uint4*>(qs);
+  void* qargs[] = {&qv, &qsv, const_cast<int*>(&rows)};
+  cudaError_t e = launch_pdl_mla(reinterpret_cast<const void*>(mla_qsplit_kernel),
+                                 dim3((n_thr + 255) / 256), dim3(256), 0, stream, qargs);
+  if (e != cudaSuccess) return e;
+  MlaScoreArgs a;
+  a.summ = static_cast<const uint8_t*>(summ);
+  a.qs = static_cast<const uint8_t*>(qs);
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.scores = scores;
+  a.status = status;
+  a.P = g.P;
+  a.max_pages = g.max_pages;
+  a.n_pool = g.n_pool;
+  const void* kern = reinterpret_cast<const void*>(score_mla_kernel);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::kSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&a};
+  const int tiles = (g.max_pages + mla::kTile - 1) / mla::kTile;
+  return launch_pdl_mla(kern, dim3(tiles, g.B), dim3(mla::kThreads), mla::kSmem, stream, args);
+}
+
+}  // namespace sa

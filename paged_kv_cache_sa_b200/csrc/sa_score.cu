@@ -447,15 +447,18 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
   float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages;
   const int tail0 = max(0, nb - a.n_tail);
   const int n_tail = a.k_cache ? nb - tail0 : 0;
-  // 1. decode-time refresh of the newest pages (overlaps the scoring grid)
-  for (int i = warp; i < n_tail; i += NT / 32) {
-    const int lp = tail0 + i;
-    const int ph = ptab_g[lp];
-    float sc = 0.f;
-    if (ph >= 0 && ph < a.n_pool)
-      sc = warp_refresh_and_score<D>(a.k_cache, a.summ, a.q + ((size_t)b * a.Hq + h * G) * D,
-                                     G, ph, h, a.Hkv, a.P, min(a.P, L - lp * a.P), lane);
-    if (lane == 0) tail_score[i] = sc;
+  // 1. decode-time refresh of the newest pages (overlaps the scoring grid).  The latent
+  //    geometry refreshes in a kernel of its own before scoring (k_cache is null here).
+  if constexpr (D <= 128) {
+    for (int i = warp; i < n_tail; i += NT / 32) {
+      const int lp = tail0 + i;
+      const int ph = ptab_g[lp];
+      float sc = 0.f;
+      if (ph >= 0 && ph < a.n_pool)
+        sc = warp_refresh_and_score<D>(a.k_cache, a.summ, a.q + ((size_t)b * a.Hq + h * G) * D,
+                                       G, ph, h, a.Hkv, a.P, min(a.P, L - lp * a.P), lane);
+      if (lane == 0) tail_score[i] = sc;
+    }
   }
   // 2. wait for the scores (one thread; the rest block on the CTA barrier)
   if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -763,19 +766,18 @@ cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
   return launch_pdl(kern, dim3(n_cta), dim3(kScoreThreads), smem, stream, args);
 }
 
-cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
-                                int n_tail, const int32_t* page_table, const int32_t* seq_lens,
-                                float* scores, int n_cta, int K, int sink_pages,
-                                int window_pages, int32_t* sel, int32_t* sel_count,
-                                int32_t* sel_phys, int32_t* status, cudaStream_t stream) {
-  cudaError_t e =
-      launch_score(g, q, summ, page_table, seq_lens, scores, n_cta, status, stream);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
+                          int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+                          float* scores, int K, int sink_pages, int window_pages, int32_t* sel,
+                          int32_t* sel_count, int32_t* sel_phys, int32_t* status,
+                          cudaStream_t stream) {
   const void* skern;
   if (g.Dk == 64)
     skern = reinterpret_cast<const void*>(select_kernel<64>);
   else if (g.Dk == 128)
     skern = reinterpret_cast<const void*>(select_kernel<128>);
+  else if (g.Dk == 576 && n_tail == 0)
+    skern = reinterpret_cast<const void*>(select_kernel<576>);
   else
     return cudaErrorInvalidValue;
   SelectArgs s;
@@ -801,12 +803,25 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
   const size_t keys_bytes = (size_t)g.max_pages * 4;
   s.ptab_in_smem = 2 * keys_bytes <= (size_t)200 * 1024;
   const size_t ssmem = s.ptab_in_smem ? 2 * keys_bytes : keys_bytes;
-  e = cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+  cudaError_t e =
+      cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(skern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   void* sargs[] = {&s};
   return launch_pdl(skern, dim3(g.Hkv, g.B), dim3(kSelectThreads), ssmem, stream, sargs);
+}
+
+cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
+                                int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+                                float* scores, int n_cta, int K, int sink_pages,
+                                int window_pages, int32_t* sel, int32_t* sel_count,
+                                int32_t* sel_phys, int32_t* status, cudaStream_t stream) {
+  cudaError_t e =
+      launch_score(g, q, summ, page_table, seq_lens, scores, n_cta, status, stream);
+  if (e != cudaSuccess) return e;
+  return launch_select(g, q, summ, k_cache, n_tail, page_table, seq_lens, scores, K, sink_pages,
+                       window_pages, sel, sel_count, sel_phys, status, stream);
 }
 
 }  // namespace sa

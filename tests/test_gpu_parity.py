@@ -183,6 +183,57 @@ def test_page_scores_alone(kw):
     assert np.allclose(got[fin], ref[fin], rtol=1e-5, atol=1e-4)
 
 
+# ------------------------------------------------------------------------------------
+# latent (MLA) geometry: 128 query heads share one 576-wide latent key per token; the
+# page scores run on the tcgen05 tensor cores
+# ------------------------------------------------------------------------------------
+
+MLA_CASES = [dict(B=2, L=(8192, 8192), seed=91),
+             dict(B=3, seq_lens=[65536, 9000, 64], seed=92),
+             dict(B=2, seq_lens=[0, 20000], seed=93, poison="nan")]
+
+
+@pytest.mark.parametrize("kw", MLA_CASES, ids=lambda kw: "-".join(
+    "%s%s" % (k, v if not isinstance(v, list) else len(v)) for k, v in kw.items()))
+def test_mla_scores_and_selection(kw):
+    case = synth.decode_case("mla", **kw)
+    dc = DevCase(case)
+    g = dc.g
+    K = case.budget // g.P
+    sa.page_summaries(g, dc.k, dc.pt, dc.sl, dc.summ)
+    ws = sa.Workspace.for_decode(g, case.budget)
+    sc = torch.full((g.B, g.Hkv, g.max_pages), 7.0, dtype=torch.float32, device="cuda")
+    sa.page_scores(g, dc.q, dc.summ, dc.pt, dc.sl, ws, scores=sc)
+    assert ws.status() == sa.SA_OK
+    summ = oracle.page_summaries(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    assert np.array_equal(u16(dc.summ), summ)
+    ref = oracle.page_scores(case.geom, case.q, summ, case.page_table, case.seq_lens)
+    got = sc.cpu().numpy()
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(got))
+    assert np.allclose(got[fin], ref[fin], rtol=1e-5, atol=1e-3), \
+        np.abs(got[fin] - ref[fin]).max()
+    # selection through the C ABI, with the newest page refreshed first
+    sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((g.B, g.Hkv), dtype=torch.int32, device="cuda")
+    phys = torch.empty_like(sel)
+    sc2 = torch.empty_like(sc)
+    sa.select_pages(g, dc.q, dc.summ, dc.pt, dc.sl, case.budget, case.sink, case.window, ws,
+                    sel=sel, sel_count=cnt, scores=sc2, k_cache=dc.k, n_tail_refresh=1,
+                    sel_phys=phys)
+    assert ws.status() == sa.SA_OK
+    assert np.array_equal(u16(dc.summ), summ)
+    osel, ocnt = oracle.select_pages(case.geom, ref, case.seq_lens, case.budget, case.sink,
+                                     case.window)
+    from parity import check_selection
+    check_selection(case.geom, case.seq_lens, case.budget, case.sink, case.window, ref, osel,
+                    ocnt, sel.cpu().numpy(), cnt.cpu().numpy())
+    gs, gc, gp = sel.cpu().numpy(), cnt.cpu().numpy(), phys.cpu().numpy()
+    for b in range(g.B):
+        c = gc[b, 0]
+        assert np.array_equal(gp[b, 0, :c], case.page_table[b, gs[b, 0, :c]])
+
+
 def test_budget_covers_all_pages_equals_dense():
     case = synth.decode_case("tiny", B=2, seq_lens=[1234, 4096], Hkv=2, Hq=8, budget=4096,
                              poison="nan")
