@@ -74,8 +74,8 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   p.off_pre = off;
   off += up256(((size_t)g.B * g.Hkv + 1) * 4);
   p.off_part = off;
-  // the latent geometry has no attention path here: no split states
-  if (!is_latent(g)) off += up256(attend_partial_floats(g, p.n_cta) * 4);
+  // split states: per warp range (GQA) or per 256-token chunk (latent)
+  off += up256(is_latent(g) ? mla_attend_part_bytes(g, p.K) : attend_partial_floats(g, p.n_cta) * 4);
   p.off_qs = off;  // latent geometry: sign-split query rows for the tensor-core scoring
   if (is_latent(g)) off += up256(mla_qsplit_bytes(g));
   p.total = off;
@@ -222,6 +222,12 @@ static int run_attend(const sa_geom& g, const DecodePlan& plan, uint8_t* w, cons
                       const int32_t* seq_lens, const int32_t* sel, const int32_t* cnt,
                       const int32_t* sel_phys, int sel_stride, float scale, float* out,
                       float* lse, cudaStream_t s) {
+  if (is_latent(g)) {
+    WsHeader* h = reinterpret_cast<WsHeader*>(w);
+    return cuda_status(launch_attend_mla(g, q, k_cache, page_table, seq_lens, sel, cnt, sel_phys,
+                                         sel_stride, scale, reinterpret_cast<float*>(w + plan.off_part),
+                                         out, lse, &h->status_bits, s));
+  }
   WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
   AttendCall c;
   c.q = q;
@@ -299,8 +305,9 @@ SA_EXPORT int sa_attend_selected(const sa_geom* g, const void* q, const void* k_
                                  size_t ws_bytes, void* stream) {
   int st = check_geom(g);
   if (st != SA_OK) return st;
-  if (!is_gqa(*g)) return SA_ERR_UNSUPPORTED;
+  if (!is_gqa(*g) && !is_latent(*g)) return SA_ERR_UNSUPPORTED;
   if (sel_stride < 1 || sel_stride > 65536) return SA_ERR_INVALID_ARG;
+  if (is_latent(*g) && !aligned16(out)) return SA_ERR_INVALID_ARG;
   if (!q || !k_cache || !page_table || !seq_lens || !sel || !sel_count || !out || !lse)
     return SA_ERR_INVALID_ARG;
   if (!g->v_aliases_k && !v_cache) return SA_ERR_INVALID_ARG;
@@ -331,7 +338,8 @@ SA_EXPORT int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_ca
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(vc) || !aligned16(summ))
     return SA_ERR_INVALID_ARG;
   if ((size_t)g->max_pages * 4 > 200 * 1024) return SA_ERR_UNSUPPORTED;
-  if (!is_gqa(*g)) return SA_ERR_UNSUPPORTED;
+  if (!is_gqa(*g) && !is_latent(*g)) return SA_ERR_UNSUPPORTED;
+  if (is_latent(*g) && !aligned16(out)) return SA_ERR_INVALID_ARG;
   DecodePlan plan;
   make_decode_plan(*g, budget, &plan);
   if (!ws || ws_bytes < plan.total || !aligned16(ws)) return SA_ERR_WORKSPACE;

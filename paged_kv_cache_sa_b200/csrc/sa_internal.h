@@ -47,6 +47,13 @@ cudaError_t launch_score_mla(const sa_geom& g, const void* q, const void* summ, 
                              const int32_t* page_table, const int32_t* seq_lens, float* scores,
                              int32_t* status, cudaStream_t stream);
 
+size_t mla_attend_part_bytes(const sa_geom& g, int sel_stride);
+cudaError_t launch_attend_mla(const sa_geom& g, const void* q, const void* kv,
+                              const int32_t* page_table, const int32_t* seq_lens,
+                              const int32_t* sel, const int32_t* sel_count,
+                              const int32_t* sel_phys, int sel_stride, float scale, float* part,
+                              float* out, float* lse, int32_t* status, cudaStream_t stream);
+
 int score_ctas(const sa_geom& g, int sms);
 bool score_supported(const sa_geom& g);
 

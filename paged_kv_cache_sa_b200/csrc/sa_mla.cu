@@ -343,4 +343,408 @@ cudaError_t launch_score_mla(const sa_geom& g, const void* q, const void* summ, 
   return launch_pdl_mla(kern, dim3(tiles, g.B), dim3(mla::kThreads), mla::kSmem, stream, args);
 }
 
+// =====================================================================================
+// Latent attention over the selected pages (tcgen05).
+//
+// Method: exact softmax attention of the 128 query heads over the tokens of the selected
+// pages, V = the first 512 channels of each token's latent row (SubQ/SSA article, SSA
+// section; Vortex summary, section 1: pages reached through the page table), split into
+// chunks of 256 tokens per CTA and merged by log-sum-exp.
+//
+// Warps 0-3 stage operands, warp 8 issues the MMAs (it must not be one of the softmax
+// warps: the P . V MMAs wait for their arrival), warps 4-7 (TMEM lane quarters 0-3) run
+// the softmax and the epilogue.
+// Per CTA (sequence b, chunk): S = Q K^T (M = 128 heads, N = 256 tokens, K = 576 in 9
+// chunks of 64 channels) accumulates in TMEM columns [0, 256); the epilogue warps (one
+// TMEM lane = one head each) take the exact softmax over the chunk and write P (bf16) to
+// shared memory in the swizzled K-major layout; O = P V (M = 128, N = 64 channels per
+// MMA, K = 256 tokens) then accumulates in TMEM columns [0, 512).  The V operand is
+// MN-major: the bytes of a token's 64-channel slice sit at the same swizzled place as the
+// K operand's chunk, so both phases use one staging routine (the second read of those
+// rows comes from L2).  The chunk's (m, l) and unnormalised O are written to the
+// workspace ([channel][head], coalesced) and attend_mla_merge_kernel combines the chunks.
+// =====================================================================================
+
+namespace mla {
+constexpr int kDv = 512;
+constexpr int kTok = 256;                       // tokens per CTA (UMMA N of Q K^T)
+constexpr int kQChunk = kG * kRowBytes;         // 16 KB: 128 head rows x 128 B
+constexpr int kKChunk = kTok * kRowBytes;       // 32 KB: 256 token rows x 128 B
+constexpr int kAStage = kQChunk + kKChunk;      // 48 KB
+constexpr int kAStages = 3;
+constexpr int kPBytes = kG * kTok * 2;          // 64 KB: P, 4 chunks of 64 tokens
+constexpr int kQkChunks = kD / kChunk;          // 9
+constexpr int kPvChunks = kDv / kChunk;         // 8
+constexpr size_t kAttnSmem = 1024 + (size_t)kAStages * kAStage + kPBytes;
+constexpr int kAttnThreads = 288;  // 4 producer, 4 softmax/epilogue, 1 MMA-issue warps
+
+// MN-major operand with 128-byte swizzle: 64 N-elements per 128-byte row, rows = K,
+// 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(32768 >> 4) << 16;  // stride between 64-element N atoms (one atom here)
+  d |= (uint64_t)(1024 >> 4) << 32;   // stride between 8-row K groups
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+}  // namespace mla
+
+struct MlaAttnArgs {
+  const uint8_t* q;        // [B][128][576] bf16
+  const uint8_t* kv;       // [n_pool][1][P][576] bf16 latent rows
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const int32_t* sel;      // [B][1][sel_stride]
+  const int32_t* sel_count;
+  const int32_t* sel_phys;  // nullable
+  float* part_o;            // [B][n_split][512][128]
+  float* part_ml;           // [B][n_split][128][2]
+  int32_t* status;
+  int P, max_pages, n_pool, sel_stride, n_split;
+  float scale_log2;
+};
+
+__global__ void __launch_bounds__(mla::kAttnThreads, 1) attend_mla_kernel(const MlaAttnArgs a) {
+  using namespace mla;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stages = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* pbuf = stages + kAStages * kAStage;  // P, 1024-aligned
+  __shared__ __align__(8) uint64_t full_bar[kAStages];
+  __shared__ __align__(8) uint64_t empty_bar[kAStages];
+  __shared__ __align__(8) uint64_t s_done, p_ready, o_done;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  __shared__ uint32_t valid_mask[kTok / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x, b = blockIdx.y;
+  const int ppc = kTok / a.P;  // pages per chunk
+
+  if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
+  const int nb = (L + a.P - 1) / a.P;
+  const int cnt = min(max(a.sel_count[b], 0), a.sel_stride);
+  const int i0 = split * ppc;
+  float* pml = a.part_ml + ((size_t)b * a.n_split + split) * kG * 2;
+  if (i0 >= cnt) {  // nothing selected in this chunk: an empty state
+    if (tid < kG) {
+      pml[tid * 2] = -INFINITY;
+      pml[tid * 2 + 1] = 0.f;
+    }
+    return;
+  }
+
+  if (tid == 0) {
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&full_bar[s], 128);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&s_done, 1);
+    mbar_init(&p_ready, 128);
+    mbar_init(&o_done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  // token rows of this chunk (producer threads r: tokens r and r + 128) and the mask of
+  // valid tokens, before the barrier that publishes it to the softmax warps
+  const uint8_t* krow[2] = {a.kv, a.kv};
+  uint32_t kbytes[2] = {0u, 0u};
+  if (warp < 4) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int t = tid + 128 * h2;
+      const int i = i0 + t / a.P;
+      const int slot = t % a.P;
+      bool ok = false;
+      int ph = 0;
+      if (i < cnt) {
+        const int lp = a.sel[(size_t)b * a.sel_stride + i];
+        if (lp >= 0 && lp < nb) {
+          ph = a.sel_phys ? a.sel_phys[(size_t)b * a.sel_stride + i]
+                          : a.page_table[(size_t)b * a.max_pages + lp];
+          if (ph < 0 || ph >= a.n_pool) {
+            report(a.status, SA_ERR_DEVICE_CHECK);
+            ph = 0;
+          } else {
+            ok = lp * a.P + slot < L;
+          }
+        }
+      }
+      krow[h2] = a.kv + ((size_t)ph * a.P + slot) * (kD * 2);
+      kbytes[h2] = ok ? 16u : 0u;  // zero-fill tokens outside the selection
+      const unsigned m = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) valid_mask[t >> 5] = m;
+    }
+  }
+  if (warp == 8) {  // all 512 TMEM columns: S in [0,256), later O in [0,512)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t st0 = smem_u32(stages);
+  const uint32_t pb0 = smem_u32(pbuf);
+
+  if (warp < 4) {
+    // ===================== producers =====================
+    // thread r: head row r of Q; token rows r and r + 128 of K/V (rows set up above)
+    const int r = tid;
+    const uint8_t* qrow = a.q + ((size_t)b * kG + r) * (kD * 2);
+    const uint32_t swz = (uint32_t)(r & 7);
+    // 9 chunks of (Q, K) for S, then 8 chunks of V (the first 512 channels) for O
+    for (int it = 0; it < kQkChunks + kPvChunks; ++it) {
+      const int s = it % kAStages;
+      if (it >= kAStages) {
+        if (!*(volatile int*)&abort_flag &&
+            !mbar_wait(&empty_bar[s], ((it / kAStages) - 1) & 1)) {
+          report(a.status, SA_ERR_TIMEOUT);
+          atomicExch(&abort_flag, 1);
+        }
+      }
+      const int kc = it < kQkChunks ? it : it - kQkChunks;
+      const uint32_t sq = st0 + s * kAStage + r * kRowBytes;
+      const uint32_t sk = st0 + s * kAStage + kQChunk;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t off = (uint32_t)((u ^ swz) << 4);
+        if (it < kQkChunks) cp_async16(sq + off, qrow + kc * kRowBytes + u * 16, 16u);
+        cp_async16(sk + r * kRowBytes + off, krow[0] + kc * kRowBytes + u * 16, kbytes[0]);
+        cp_async16(sk + (r + 128) * kRowBytes + off, krow[1] + kc * kRowBytes + u * 16,
+                   kbytes[1]);
+      }
+      cp_async_commit();
+      if (it >= kAStages - 1) {
+        cp_async_wait<kAStages - 1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&full_bar[(it - (kAStages - 1)) % kAStages]);
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    for (int it = kQkChunks + kPvChunks - (kAStages - 1); it < kQkChunks + kPvChunks; ++it)
+      mbar_arrive(&full_bar[it % kAStages]);
+  } else if (warp == 8) {
+    // ===================== MMA issue (one thread of its own warp) =====================
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(kG, kTok);
+      constexpr uint32_t idesc_o = idesc_bf16(kG, 64) | (1u << 16);  // B (V) MN-major
+      bool ok = true;
+      for (int it = 0; it < kQkChunks + kPvChunks && ok; ++it) {
+        const int s = it % kAStages;
+        if (it == kQkChunks) {
+          umma_commit(&s_done);  // S complete -> softmax
+          if (!mbar_wait(&p_ready, 0)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (*(volatile int*)&abort_flag || !mbar_wait(&full_bar[s], (it / kAStages) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sq = st0 + s * kAStage;
+        const uint32_t sk = sq + kQChunk;
+        if (it < kQkChunks) {
+#pragma unroll
+          for (int k = 0; k < kChunk / 16; ++k)
+            umma_bf16(tmem, desc_sw128(sq + k * 32), desc_sw128(sk + k * 32), idesc_s,
+                      (it | k) != 0);
+        } else {
+          const int cb = it - kQkChunks;  // channels 64*cb .. 64*cb + 63
+#pragma unroll 4
+          for (int kk = 0; kk < kTok / 16; ++kk)
+            umma_bf16(tmem + 64 * cb,
+                      desc_sw128(pb0 + (kk >> 2) * (kG * kRowBytes) + (kk & 3) * 32),
+                      desc_sw128_mn(sk + kk * 16 * kRowBytes), idesc_o, kk != 0);
+        }
+        umma_commit(&empty_bar[s]);
+      }
+      if (!ok) {
+        report(a.status, SA_ERR_TIMEOUT);
+        atomicExch(&abort_flag, 1);
+        umma_commit(&s_done);  // never leave the epilogue waiting (bounded anyway)
+      }
+      umma_commit(&o_done);
+    }
+    __syncwarp();
+  } else {
+    const int wq = warp - 4;  // TMEM lanes 32*wq .. : heads 32*wq + lane
+    const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
+    // ===================== softmax over the chunk (one head per thread) ==========
+    const int head = 32 * wq + lane;
+    bool ready = __all_sync(0xffffffffu, mbar_wait(&s_done, 0));
+    tc_fence_after();
+    float m = -INFINITY, l = 0.f;
+    if (ready) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTok; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + c0, v);
+        const uint32_t vm = valid_mask[c0 >> 5];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if ((vm >> i) & 1) m = fmaxf(m, v[i] * a.scale_log2);
+      }
+      // P = 2^(x - m) in bf16, K-major swizzled rows (row = head), and l = sum of P
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTok; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + c0, v);
+        const uint32_t vm = valid_mask[c0 >> 5];
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ((vm >> (2 * i)) & 1) ? fast_exp2(v[2 * i] * a.scale_log2 - m) : 0.f;
+          const float p1 =
+              ((vm >> (2 * i + 1)) & 1) ? fast_exp2(v[2 * i + 1] * a.scale_log2 - m) : 0.f;
+          l += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        // tokens c0 .. c0+31 = chunk c0/64, 16-byte units (c0 % 64)/8 .. +3
+        const uint32_t rowp = pb0 + (c0 >> 6) * (kG * kRowBytes) + head * kRowBytes;
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const int u = ((c0 & 63) >> 3) + u4;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           rowp + ((u ^ (head & 7)) << 4)),
+                       "r"(pk[4 * u4]), "r"(pk[4 * u4 + 1]), "r"(pk[4 * u4 + 2]),
+                       "r"(pk[4 * u4 + 3])
+                       : "memory");
+        }
+      }
+    }
+    fence_proxy_async_smem();  // P (generic stores) -> tensor-core reads
+    tc_fence_before();
+    mbar_arrive(&p_ready);
+    // ===================== O epilogue: the chunk's state to the workspace ==========
+    ready = __all_sync(0xffffffffu, mbar_wait(&o_done, 0)) && ready;
+    tc_fence_after();
+    const bool good = ready && !*(volatile int*)&abort_flag;
+    float* po = a.part_o + ((size_t)b * a.n_split + split) * kDv * kG;
+    if (good) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < kDv; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + c0, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) po[(size_t)(c0 + i) * kG + head] = v[i];
+      }
+    } else if (lane == 0) {
+      report(a.status, SA_ERR_TIMEOUT);
+    }
+    pml[head * 2] = good ? m : -INFINITY;
+    pml[head * 2 + 1] = good ? l : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+// Combine the chunk states of each (sequence, head): out = sum_s 2^(m_s - M) O_s / L,
+// lse = (M + log2 L) ln 2.  CTA = (sequence, 32 channels); thread = head.
+__global__ void __launch_bounds__(128) attend_mla_merge_kernel(const float* __restrict__ part_o,
+                                                               const float* __restrict__ part_ml,
+                                                               float* __restrict__ out,
+                                                               float* __restrict__ lse,
+                                                               int n_split) {
+  using namespace mla;
+  __shared__ float tile[kG][33];
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int b = blockIdx.y, c0 = blockIdx.x * 32, h = threadIdx.x;
+  const float* ml = part_ml + (size_t)b * n_split * kG * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < n_split; ++s) M = fmaxf(M, ml[((size_t)s * kG + h) * 2]);
+  float Lsum = 0.f, acc[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    const float ms = ml[((size_t)s * kG + h) * 2];
+    if (ms == -INFINITY) continue;
+    const float w = fast_exp2(ms - M);
+    Lsum += w * ml[((size_t)s * kG + h) * 2 + 1];
+    const float* po = part_o + (((size_t)b * n_split + s) * kDv + c0) * kG + h;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] += w * po[(size_t)i * kG];
+  }
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) tile[h][i] = acc[i] * inv;
+  if (blockIdx.x == 0)
+    lse[(size_t)b * kG + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+  __syncthreads();
+  // write rows out[b][h][c0 .. c0+31]: 8 threads per head row, 4 floats each
+  for (int e = h; e < kG * 8; e += 128) {
+    const int hh = e >> 3, q4 = (e & 7) * 4;
+    *reinterpret_cast<float4*>(out + ((size_t)b * kG + hh) * kDv + c0 + q4) =
+        make_float4(tile[hh][q4], tile[hh][q4 + 1], tile[hh][q4 + 2], tile[hh][q4 + 3]);
+  }
+}
+
+int mla_attend_splits(const sa_geom& g, int sel_stride) {
+  const int ppc = mla::kTok / g.P;
+  return (sel_stride + ppc - 1) / ppc;
+}
+
+size_t mla_attend_part_bytes(const sa_geom& g, int sel_stride) {
+  const size_t ns = (size_t)mla_attend_splits(g, sel_stride);
+  return (size_t)g.B * ns * mla::kG * (mla::kDv + 2) * 4;
+}
+
+cudaError_t launch_attend_mla(const sa_geom& g, const void* q, const void* kv,
+                              const int32_t* page_table, const int32_t* seq_lens,
+                              const int32_t* sel, const int32_t* sel_count,
+                              const int32_t* sel_phys, int sel_stride, float scale, float* part,
+                              float* out, float* lse, int32_t* status, cudaStream_t stream) {
+  MlaAttnArgs a;
+  a.q = static_cast<const uint8_t*>(q);
+  a.kv = static_cast<const uint8_t*>(kv);
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.sel = sel;
+  a.sel_count = sel_count;
+  a.sel_phys = sel_phys;
+  a.n_split = mla_attend_splits(g, sel_stride);
+  a.part_o = part;
+  a.part_ml = part + (size_t)g.B * a.n_split * mla::kDv * mla::kG;
+  a.status = status;
+  a.P = g.P;
+  a.max_pages = g.max_pages;
+  a.n_pool = g.n_pool;
+  a.sel_stride = sel_stride;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const void* kern = reinterpret_cast<const void*>(attend_mla_kernel);
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::kAttnSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&a};
+  e = launch_pdl_mla(kern, dim3(a.n_split, g.B), dim3(mla::kAttnThreads), mla::kAttnSmem,
+                     stream, args);
+  if (e != cudaSuccess) return e;
+  const float* po = a.part_o;
+  const float* pml = a.part_ml;
+  int ns = a.n_split;
+  void* margs[] = {&po, &pml, &out, &lse, &ns};
+  return launch_pdl_mla(reinterpret_cast<const void*>(attend_mla_merge_kernel),
+                        dim3(mla::kDv / 32, g.B), dim3(128), 0, stream, margs);
+}
+
 }  // namespace sa

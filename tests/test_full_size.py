@@ -18,7 +18,7 @@ from parity import DevCase, check_attention, check_selection, u16
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("wl", ["llama32k", "llama128k"])
+@pytest.mark.parametrize("wl", ["llama32k", "llama128k", "mla"])
 def test_full_size_bench_launch_config(wl):
     import torch
     import paged_kv_cache_sa_b200 as sa

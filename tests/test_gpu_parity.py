@@ -234,6 +234,29 @@ def test_mla_scores_and_selection(kw):
         assert np.array_equal(gp[b, 0, :c], case.page_table[b, gs[b, 0, :c]])
 
 
+@pytest.mark.parametrize("kw", MLA_CASES + [dict(B=2, seq_lens=[65536, 4000], seed=94,
+                                                  budget=4096, sink=64, window=1024)],
+                         ids=lambda kw: "-".join("%s%s" % (k, v if not isinstance(v, list)
+                                                           else len(v)) for k, v in kw.items()))
+def test_mla_decode_parity(kw):
+    # scores + selection + tensor-core attention over the latent rows (V = first 512)
+    case = synth.decode_case("mla", **kw)
+    res = run_decode(DevCase(case))
+    full_parity(case, res)
+
+
+def test_mla_budget_covers_all_pages_equals_dense():
+    case = synth.decode_case("mla", B=2, seq_lens=[1500, 777], budget=1536, seed=95)
+    res = run_decode(DevCase(case))
+    g = case.geom
+    for b in range(g.B):
+        L = int(case.seq_lens[b])
+        rows = np.concatenate([case.k_cache[case.page_table[b, p], 0]
+                               for p in range((L + g.P - 1) // g.P)])[:L]
+        o, l = oracle.dense_attend(case.q[b], rows, rows[:, :g.Dv], case.scale)
+        check_attention(res["out"][b], res["lse"][b], o, l)
+
+
 def test_budget_covers_all_pages_equals_dense():
     case = synth.decode_case("tiny", B=2, seq_lens=[1234, 4096], Hkv=2, Hq=8, budget=4096,
                              poison="nan")
