@@ -43,7 +43,7 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 N_LAYERS = 32
-WORKLOADS = ("llama32k", "llama128k", "ragged")
+WORKLOADS = ("llama32k", "llama128k", "ragged", "mla")
 
 
 def parse():
@@ -227,14 +227,16 @@ def run_native(args, rank, world, dist):
     L_layers = args.layers
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16
                                                           else a)).to(dev)
-    k0, v0 = t(case.k_cache), t(case.v_cache)
+    k0 = t(case.k_cache)
+    v0 = t(case.v_cache) if case.v_cache is not None else None  # latent: V aliases K
     pt, sl = t(case.page_table), t(case.seq_lens)
     rng = np.random.default_rng(1234 + rank)
     ks, vs, qs, summs = [], [], [], []
     stride = max(1, g.n_pool // L_layers)
     for l in range(L_layers):
         ks.append(k0 if l == 0 else torch.roll(k0, shifts=l * stride, dims=0))
-        vs.append(v0 if l == 0 else torch.roll(v0, shifts=l * stride, dims=0))
+        vs.append(None if v0 is None else
+                  (v0 if l == 0 else torch.roll(v0, shifts=l * stride, dims=0)))
         qn = case.q if l == 0 else synth.f32_to_bf16(rng.standard_normal(case.q.shape).astype(np.float32))
         qs.append(t(qn))
         summs.append(torch.empty((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device=dev))
@@ -388,12 +390,15 @@ def run_native(args, rank, world, dist):
     sel_mean = float(sel_ms.mean())
     sc_mean = float(sc_ms.mean())
     # page scoring: summaries + page-table entries + queries of one layer per launch
-    dom_kernel, dom_bytes, dom_ms = "score_stream_kernel", sel_b, sc_mean
+    dom_kernel = "score_mla_kernel" if g.v_aliases_k else "score_stream_kernel"
+    dom_bytes, dom_ms = sel_b, sc_mean
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     cpu_v, cpu_done, cpu_t = (None, 0, 0.0)
     if world == 1:
         cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds)
-    launches_per_layer = 4  # score, select (+ tail refresh), attention, merge
+    # GQA: score, select (+ tail refresh), attention, merge; latent: tail refresh, query
+    # sign split, tensor-core score, select, tensor-core attention, merge
+    launches_per_layer = 6 if g.v_aliases_k else 4
     line = {
         "metric": "sparse-decode seq*heads/s",
         "value": value,
@@ -422,6 +427,7 @@ def run_native(args, rank, world, dist):
             "attend_selected_us_alone": att_mean * 1e3,
             "page_scores_us_alone": sc_mean * 1e3,
             "algorithmic_bytes_per_layer": sel_b + att_b + upd_b,
+            **mla_flops(case, sel_count, sc_mean, att_mean),
         },
         "roofline": {
             "kernel": dom_kernel,
@@ -441,6 +447,27 @@ def run_native(args, rank, world, dist):
     }
     print(json.dumps(line, default=_json_default), flush=True)
     return 0
+
+
+def mla_flops(case, sel_count, score_ms, attend_ms):
+    """Latent geometry: tensor-core work per layer (scores as a GEMM over 2*Dk, Q.K^T
+    and P.V over the selected tokens) and its rate in the timed-alone phases."""
+    g = case.geom
+    if not g.v_aliases_k:
+        return {}
+    P = g.P
+    nb = (case.seq_lens.astype(np.int64) + P - 1) // P
+    score_f = 2.0 * g.Hq * 2 * g.Dk * float(nb.sum())
+    tok = 0
+    for b in range(g.B):
+        L = int(case.seq_lens[b])
+        last = L - (int(nb[b]) - 1) * P if nb[b] else 0
+        c = int(sel_count[b, 0])
+        tok += c * P - (P - last if c else 0)
+    att_f = 2.0 * g.Hq * (g.Dk + g.Dv) * tok
+    return {"score_gflop_per_layer": score_f / 1e9, "attend_gflop_per_layer": att_f / 1e9,
+            "score_tflops_alone": score_f / (score_ms * 1e-3) / 1e12,
+            "attend_tflops_alone": att_f / (attend_ms * 1e-3) / 1e12}
 
 
 def recorded_traffic(kernel, workload):

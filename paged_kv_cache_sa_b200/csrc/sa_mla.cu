@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1) score_mla_kernel(const MlaSc
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
+  __shared__ int row_ph[mla::kTile];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile = blockIdx.x, b = blockIdx.y;
   const int p0 = tile * kTile;
@@ -182,6 +183,18 @@ __global__ void __launch_bounds__(mla::kThreads, 1) score_mla_kernel(const MlaSc
     abort_flag = 0;
     fence_mbar_init();
   }
+  if (tid < kTile) {  // physical page of every row of the tile (-1: zero row)
+    const int p = p0 + tid;
+    int ph = -1;
+    if (p < nb) {
+      ph = a.page_table[(size_t)b * a.max_pages + p];
+      if (ph < 0 || ph >= a.n_pool) {
+        report(a.status, SA_ERR_DEVICE_CHECK);
+        ph = -1;
+      }
+    }
+    row_ph[tid] = ph;
+  }
   if (warp == 4) {  // TMEM: 128 fp32 columns (one per head), 128 lanes (one per page)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&tmem_base)),
@@ -197,21 +210,10 @@ __global__ void __launch_bounds__(mla::kThreads, 1) score_mla_kernel(const MlaSc
 
   if (warp < 4) {
     // ===================== producers: 16-byte copies into swizzled stages ==========
-    // thread r owns row r of both operands: page p0 + r of A, head r of B
-    const int r = tid;
-    const int p = p0 + r;
-    int ph = -1;
-    if (p < nb) {
-      ph = a.page_table[(size_t)b * a.max_pages + p];
-      if (ph < 0 || ph >= a.n_pool) {
-        report(a.status, SA_ERR_DEVICE_CHECK);
-        ph = -1;
-      }
-    }
-    const uint8_t* arow = a.summ + (size_t)(ph < 0 ? 0 : ph) * (kK * 2);
-    const uint32_t asrc_bytes = ph < 0 ? 0u : 16u;  // zero-fill rows outside the sequence
-    const uint8_t* brow = a.qs + ((size_t)b * kG + r) * (kK * 2);
-    const uint32_t swz = (uint32_t)(r & 7);
+    // eight consecutive lanes copy one 128-byte row of a chunk (coalesced); a warp covers
+    // four rows per pass, the four producer warps 16 rows, eight passes the 128 rows
+    const int u = lane & 7;
+    const int rsub = warp * 4 + (lane >> 3);
     for (int kc = 0; kc < kChunks; ++kc) {
       const int s = kc % kStages;
       if (kc >= kStages) {
@@ -221,13 +223,17 @@ __global__ void __launch_bounds__(mla::kThreads, 1) score_mla_kernel(const MlaSc
           atomicExch(&abort_flag, 1);
         }
       }
-      const uint32_t sa_ = st0 + s * kStageBytes + r * kRowBytes;
-      const uint32_t sb_ = sa_ + kOpBytes;
+      const uint32_t sa_ = st0 + s * kStageBytes;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t off = (uint32_t)((u ^ swz) << 4);
-        cp_async16(sa_ + off, arow + kc * kRowBytes + u * 16, asrc_bytes);
-        cp_async16(sb_ + off, brow + kc * kRowBytes + u * 16, 16u);
+      for (int i = 0; i < kTile / 16; ++i) {
+        const int r = 16 * i + rsub;
+        const int ph = row_ph[r];
+        const uint32_t off = (uint32_t)(r * kRowBytes + ((u ^ (r & 7)) << 4));
+        // rows outside the sequence are zero-filled (source size 0)
+        cp_async16(sa_ + off, a.summ + (size_t)(ph < 0 ? 0 : ph) * (kK * 2) + kc * kRowBytes + u * 16,
+                   ph < 0 ? 0u : 16u);
+        cp_async16(sa_ + kOpBytes + off,
+                   a.qs + ((size_t)b * kG + r) * (kK * 2) + kc * kRowBytes + u * 16, 16u);
       }
       cp_async_commit();
       // the stage issued kStages-1 chunks ago has landed: publish it to the MMA thread
@@ -418,6 +424,7 @@ __global__ void __launch_bounds__(mla::kAttnThreads, 1) attend_mla_kernel(const 
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   __shared__ uint32_t valid_mask[kTok / 32];
+  __shared__ int tok_row[kTok];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, b = blockIdx.y;
   const int ppc = kTok / a.P;  // pages per chunk
@@ -449,34 +456,29 @@ __global__ void __launch_bounds__(mla::kAttnThreads, 1) attend_mla_kernel(const 
     abort_flag = 0;
     fence_mbar_init();
   }
-  // token rows of this chunk (producer threads r: tokens r and r + 128) and the mask of
-  // valid tokens, before the barrier that publishes it to the softmax warps
-  const uint8_t* krow[2] = {a.kv, a.kv};
-  uint32_t kbytes[2] = {0u, 0u};
+  // token rows of this chunk (thread r: tokens r and r + 128): latent row index in the
+  // pool (-1: zero row) and the mask of valid tokens, before the barrier that publishes
+  // them to the producers and the softmax warps
   if (warp < 4) {
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       const int t = tid + 128 * h2;
       const int i = i0 + t / a.P;
       const int slot = t % a.P;
-      bool ok = false;
-      int ph = 0;
+      int row = -1;
       if (i < cnt) {
         const int lp = a.sel[(size_t)b * a.sel_stride + i];
         if (lp >= 0 && lp < nb) {
-          ph = a.sel_phys ? a.sel_phys[(size_t)b * a.sel_stride + i]
-                          : a.page_table[(size_t)b * a.max_pages + lp];
-          if (ph < 0 || ph >= a.n_pool) {
+          const int ph = a.sel_phys ? a.sel_phys[(size_t)b * a.sel_stride + i]
+                                    : a.page_table[(size_t)b * a.max_pages + lp];
+          if (ph < 0 || ph >= a.n_pool)
             report(a.status, SA_ERR_DEVICE_CHECK);
-            ph = 0;
-          } else {
-            ok = lp * a.P + slot < L;
-          }
+          else if (lp * a.P + slot < L)
+            row = ph * a.P + slot;
         }
       }
-      krow[h2] = a.kv + ((size_t)ph * a.P + slot) * (kD * 2);
-      kbytes[h2] = ok ? 16u : 0u;  // zero-fill tokens outside the selection
-      const unsigned m = __ballot_sync(0xffffffffu, ok);
+      tok_row[t] = row;
+      const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
       if (lane == 0) valid_mask[t >> 5] = m;
     }
   }
@@ -496,10 +498,10 @@ __global__ void __launch_bounds__(mla::kAttnThreads, 1) attend_mla_kernel(const 
 
   if (warp < 4) {
     // ===================== producers =====================
-    // thread r: head row r of Q; token rows r and r + 128 of K/V (rows set up above)
-    const int r = tid;
-    const uint8_t* qrow = a.q + ((size_t)b * kG + r) * (kD * 2);
-    const uint32_t swz = (uint32_t)(r & 7);
+    // eight consecutive lanes copy one 128-byte row of a chunk (coalesced): 8 passes of
+    // 16 rows for the 128 query rows, 16 passes for the 256 token rows
+    const int u = lane & 7;
+    const int rsub = warp * 4 + (lane >> 3);
     // 9 chunks of (Q, K) for S, then 8 chunks of V (the first 512 channels) for O
     for (int it = 0; it < kQkChunks + kPvChunks; ++it) {
       const int s = it % kAStages;
@@ -511,15 +513,24 @@ __global__ void __launch_bounds__(mla::kAttnThreads, 1) attend_mla_kernel(const 
         }
       }
       const int kc = it < kQkChunks ? it : it - kQkChunks;
-      const uint32_t sq = st0 + s * kAStage + r * kRowBytes;
-      const uint32_t sk = st0 + s * kAStage + kQChunk;
+      const uint32_t sq = st0 + s * kAStage;
+      const uint32_t sk = sq + kQChunk;
+      if (it < kQkChunks) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t off = (uint32_t)((u ^ swz) << 4);
-        if (it < kQkChunks) cp_async16(sq + off, qrow + kc * kRowBytes + u * 16, 16u);
-        cp_async16(sk + r * kRowBytes + off, krow[0] + kc * kRowBytes + u * 16, kbytes[0]);
-        cp_async16(sk + (r + 128) * kRowBytes + off, krow[1] + kc * kRowBytes + u * 16,
-                   kbytes[1]);
+        for (int i = 0; i < kG / 16; ++i) {
+          const int r = 16 * i + rsub;
+          cp_async16(sq + r * kRowBytes + ((u ^ (r & 7)) << 4),
+                     a.q + ((size_t)b * kG + r) * (kD * 2) + kc * kRowBytes + u * 16, 16u);
+        }
+      }
+#pragma unroll 4
+      for (int i = 0; i < kTok / 16; ++i) {
+        const int t = 16 * i + rsub;
+        const int row = tok_row[t];
+        // tokens outside the selection are zero-filled (source size 0)
+        cp_async16(sk + t * kRowBytes + ((u ^ (t & 7)) << 4),
+                   a.kv + (size_t)(row < 0 ? 0 : row) * (kD * 2) + kc * kRowBytes + u * 16,
+                   row < 0 ? 0u : 16u);
       }
       cp_async_commit();
       if (it >= kAStages - 1) {
