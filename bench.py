@@ -43,7 +43,7 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 N_LAYERS = 32
-WORKLOADS = ("llama32k", "llama128k", "ragged", "mla")
+WORKLOADS = ("llama32k", "llama128k", "ragged", "mla", "tiny")
 
 
 def parse():
@@ -76,6 +76,27 @@ def peaks():
 # ------------------------------------------------------------------------------------
 # algorithmic bytes (inherent to the method; workspace traffic excluded)
 # ------------------------------------------------------------------------------------
+
+def rank_seed(workload, rank):
+    """Seed of rank `rank`'s batch: every rank decodes its own sequences (replicas)."""
+    return synth.WORKLOADS[workload]["seed"] + 1000 * rank
+
+
+def max_over_ranks(x, dist, device="cpu"):
+    """The largest of the ranks' values of `x` (a duration): the job ends with its slowest
+    rank.  `dist` is torch.distributed (or None for one process)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step, world, ms_per_step):
+    """Units per second of the whole job: every rank processes its own units per step."""
+    return units_per_rank_step * world / (ms_per_step * 1e-3)
+
 
 def layer_bytes(geom, seq_lens, sel_count, P):
     """Per layer-call: (select_bytes, attend_bytes, update_bytes)."""
@@ -221,7 +242,7 @@ def run_native(args, rank, world, dist):
 
     # ---- inputs: layer 0 from the seeded generator (rank-specific seed), other layers
     # are the same bytes rolled along the page axis (distinct memory and content)
-    case = synth.decode_case(args.workload, seed=synth.WORKLOADS[args.workload]["seed"] + 1000 * rank)
+    case = synth.decode_case(args.workload, seed=rank_seed(args.workload, rank))
     g = Geometry.of(case.geom)
     P = g.P
     L_layers = args.layers
@@ -324,14 +345,10 @@ def run_native(args, rank, world, dist):
     torch.cuda.synchronize()
     total_ms = t0e.elapsed_time(t1e)
     clk = clocks.stop()
-    if dist is not None:
-        import torch.distributed as tdist
-        tt = torch.tensor([total_ms], device=dev)
-        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_ms / args.steps
     units_per_step = g.B * g.Hq * L_layers
-    value = units_per_step * world / (ms_per_step * 1e-3)
+    value = whole_job_rate(units_per_step, world, ms_per_step)
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
     # ---- per-phase durations (events on the launching stream), averaged over replays
@@ -375,11 +392,7 @@ def run_native(args, rank, world, dist):
         e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist is not None:
-        import torch.distributed as tdist
-        tt = torch.tensor([e2e_ms], device=dev)
-        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     assert ws.status() == sa.SA_OK
     h2d = sum(int(x.numel()) * 2 for x in q_host)
     d2h = sum(int(x.numel()) * 4 for x in o_host) + sum(int(x.numel()) * 4 for x in l_host)
@@ -440,7 +453,7 @@ def run_native(args, rank, world, dist):
             "value": cpu_v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
             "sample": "%d (sequence, layer) decode calls of layer 0 (score+select+attend over "
                       "all %d query heads), %.1f s single-threaded" % (cpu_done, g.Hq, cpu_t)},
-        "e2e": {"value": units_per_step * world / (e2e_ms * 1e-3), "unit": "seq*heads/s",
+        "e2e": {"value": whole_job_rate(units_per_step, world, e2e_ms), "unit": "seq*heads/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_layer * L_layers * args.steps,
         "clocks": clk,
@@ -500,7 +513,9 @@ def main():
         import datetime
         import torch
         import torch.distributed as tdist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        if args.impl == "native":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        # the native arm's ranks time GPUs (NCCL); the oracle arm runs on host cores (gloo)
         tdist.init_process_group("nccl" if args.impl == "native" else "gloo",
                                  timeout=datetime.timedelta(seconds=300))
         dist = tdist
