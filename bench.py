@@ -2,12 +2,12 @@
 
 One step = one decode step of a 32-layer model with Llama-3.1-8B attention geometry
 (batch 8, 32 query / 8 KV heads, head dim 128, 32768 tokens per sequence, page 16,
-token budget 2048 = sink 64 + window 512 + top-k).  Per layer, sa_select_pages scores
-every page against the query (streaming kernel) and selects the top pages (per-pair
-select kernel, which also refreshes the summary of each sequence's newest page), then
-sa_attend_selected runs split-KV attention over the gathered pages (attention kernel
-plus the merge kernel of the pairs split across warps) -- the two halves of
-sa_sparse_decode.  Every layer owns its own KV pool, so a step touches ~4.3 GB (> L2)
+token budget 2048 = sink 64 + window 512 + top-k).  Per layer, one sa_sparse_decode call
+scores every page against the query (streaming kernel), selects the top pages (per-pair
+select kernel, which also refreshes the summary of each sequence's newest page) and runs
+split-KV attention over the gathered pages
+(attention kernel plus the merge kernel of the pairs split across warps).  Its two
+halves, sa_select_pages and sa_attend_selected, are timed apart for context.  Every layer owns its own KV pool, so a step touches ~4.3 GB (> L2)
 and nothing is served from L2 across layers.
 
 Metric: sparse-decode seq*heads/s = (sequence, query head) attention outputs of one
@@ -274,6 +274,13 @@ def run_native(args, rank, world, dist):
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
           for _ in range(L_layers)]
 
+    def step_fused():
+        # the headline: one sa_sparse_decode per layer (selection + attention)
+        for l in range(L_layers):
+            sa.sparse_decode(g, qs[l], ks[l], vs[l], summs[l], pt, sl, case.budget, case.sink,
+                             case.window, case.scale, ws, out=outs[l], lse=lses[l],
+                             sel_out=sel, sel_count_out=cnt, n_tail_refresh=1)
+
     def step(with_events):
         for l in range(L_layers):
             if with_events:
@@ -289,7 +296,7 @@ def run_native(args, rank, world, dist):
                 ev[l][2].record()
 
     # one eager step: correctness of the launch config, selection counts for the bytes
-    step(False)
+    step_fused()
     assert ws.status() == sa.SA_OK
     sel_count = cnt.cpu().numpy()
     sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, P)
@@ -315,10 +322,11 @@ def run_native(args, rank, world, dist):
     graph_sc = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         step(True)                      # warm the stream before capture
+        step_fused()
         score_only()
         torch.cuda.synchronize()
         with torch.cuda.graph(graph, stream=stream):
-            step(False)
+            step_fused()
         with torch.cuda.graph(graph_ev, stream=stream):
             step(True)
         with torch.cuda.graph(graph_sc, stream=stream):
