@@ -43,7 +43,7 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 N_LAYERS = 32
-WORKLOADS = ("llama32k", "llama128k", "ragged", "mla", "tiny")
+WORKLOADS = ("llama32k", "llama128k", "ragged", "mla", "tiny", "prune")
 
 
 def parse():
@@ -262,6 +262,18 @@ def run_native(args, rank, world, dist):
         qs.append(t(qn))
         summs.append(torch.empty((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device=dev))
         sa.page_summaries(g, ks[l], pt, sl, summs[l])
+    # per-page summaries (row a-1) of one layer's pool, timed alone: K read once
+    e_s0, e_s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e_s0.record()
+    for _ in range(3):
+        sa.page_summaries(g, ks[0], pt, sl, summs[0])
+    e_s1.record()
+    torch.cuda.synchronize()
+    summ_ms = e_s0.elapsed_time(e_s1) / 3
+    n_used = int(((case.seq_lens.astype(np.int64) + P - 1) // P).sum())
+    summ_bytes = int(case.seq_lens.astype(np.int64).sum()) * g.Hkv * g.Dk * 2 + \
+        n_used * g.Hkv * 2 * g.Dk * 2 + n_used * 4
     K = case.budget // P
     ws = sa.Workspace.for_decode(g, case.budget)
     sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device=dev)
@@ -447,6 +459,8 @@ def run_native(args, rank, world, dist):
             "select_pages_us_alone": sel_mean * 1e3,
             "attend_selected_us_alone": att_mean * 1e3,
             "page_scores_us_alone": sc_mean * 1e3,
+            "summaries_us_alone": summ_ms * 1e3,
+            "summaries_gbs_alone": summ_bytes / (summ_ms * 1e-3) / 1e9,
             "algorithmic_bytes_per_layer": sel_b + att_b + upd_b,
             **mla_flops(case, sel_count, sc_mean, att_mean),
         },
@@ -491,6 +505,193 @@ def mla_flops(case, sel_count, score_ms, attend_ms):
             "attend_tflops_alone": att_f / (attend_ms * 1e-3) / 1e12}
 
 
+# ------------------------------------------------------------------------------------
+# prune workload: compaction of every session, then one decode over the compacted cache
+# ------------------------------------------------------------------------------------
+
+def prune_bytes(case, keep):
+    """Algorithmic bytes of one compaction: kept tokens read and written (K and V, every
+    KV head), the keep-mask, the new pages' summaries and tables."""
+    g = case.geom
+    kept = 0
+    pages = 0
+    for b in range(g.B):
+        L = int(case.seq_lens[b])
+        k = int(keep[b, :L].sum())
+        kept += k
+        pages += (k + g.P - 1) // g.P
+    row = g.Hkv * (g.Dk + (0 if g.v_aliases_k else g.Dv)) * 2
+    mask = int(case.seq_lens.sum())
+    return 2 * kept * row + mask + pages * g.Hkv * 2 * g.Dk * 2 + g.B * g.max_pages * 4, kept
+
+
+def oracle_prune_sample(pc, seconds):
+    """Time the CPU oracle's compaction session by session until ~`seconds` elapsed."""
+    import oracle
+    d = pc.decode
+    g = d.geom
+    done, t_total, b = 0, 0.0, 0
+    fp_off = 0
+    while t_total < seconds and done < g.B:
+        sub = synth.Geometry(1, g.Hq, g.Hkv, g.Dk, g.Dv, g.P, g.max_pages, g.n_pool, g.v_aliases_k)
+        L = int(d.seq_lens[b])
+        need = (int(pc.keep[b, :L].sum()) + g.P - 1) // g.P
+        t0 = time.perf_counter()
+        oracle.prune_compact(sub, d.k_cache, d.v_cache, d.page_table[b:b + 1], d.seq_lens[b:b + 1],
+                             pc.keep[b:b + 1], pc.free_pages[fp_off:fp_off + need])
+        t_total += time.perf_counter() - t0
+        fp_off += need
+        done += 1
+        b += 1
+    return done / t_total, done, t_total
+
+
+def run_prune(args, rank, world, dist):
+    import torch
+    import paged_kv_cache_sa_b200 as sa
+    from paged_kv_cache_sa_b200 import Geometry
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    hbm_peak, _, peak_kind = peaks()
+    pc = synth.prune_case("prune", seed=rank_seed("prune", rank))
+    d = pc.decode
+    g = Geometry.of(d.geom)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16
+                                                          else a)).to(dev)
+    k, v = t(d.k_cache), t(d.v_cache)
+    pt, sl, keep, fp = t(d.page_table), t(d.seq_lens), t(pc.keep), t(pc.free_pages)
+    q = t(d.q)
+    summ = torch.zeros((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device=dev)
+    wsp = sa.Workspace.for_prune(g)
+    wsd = sa.Workspace.for_decode(g, d.budget)
+    width = g.max_pages * g.P
+    npt = torch.empty((g.B, g.max_pages), dtype=torch.int32, device=dev)
+    nsl = torch.empty((g.B,), dtype=torch.int32, device=dev)
+    pos = torch.empty((g.B, width), dtype=torch.int32, device=dev)
+    ll = torch.empty((g.B,), dtype=torch.int32, device=dev)
+    out = torch.empty((g.B, g.Hq, g.Dv), dtype=torch.float32, device=dev)
+    lse = torch.empty((g.B, g.Hq), dtype=torch.float32, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+
+    def step(with_events):
+        # compaction into the fresh pages (the old pages stay readable: repeating the
+        # step rewrites the same bytes), then one decode over the compacted cache
+        if with_events:
+            ev[0].record()
+        sa.prune_compact(g, k, v, pt, sl, keep, fp, k, v, summ, wsp, new_page_table=npt,
+                         new_seq_lens=nsl, pos_map=pos, logical_len=ll)
+        if with_events:
+            ev[1].record()
+        sa.sparse_decode(g, q, k, v, summ, npt, nsl, d.budget, d.sink, d.window, d.scale, wsd,
+                         out=out, lse=lse)
+        if with_events:
+            ev[2].record()
+
+    step(False)
+    torch.cuda.synchronize()
+    assert wsp.status() == sa.SA_OK and wsd.status() == sa.SA_OK
+    pbytes, kept = prune_bytes(d, pc.keep)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph, graph_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        step(True)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            step(False)
+        with torch.cuda.graph(graph_ev, stream=stream):
+            step(True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0e.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        t1e.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms_per_step = max_over_ranks(t0e.elapsed_time(t1e), dist, dev) / args.steps
+    prune_ms = dec_ms = 0.0
+    n_ev = max(3, args.steps // 2)
+    with torch.cuda.stream(stream):
+        for _ in range(n_ev):
+            graph_ev.replay()
+            torch.cuda.synchronize()
+            prune_ms += ev[0].elapsed_time(ev[1]) / n_ev
+            dec_ms += ev[1].elapsed_time(ev[2]) / n_ev
+    assert wsp.status() == sa.SA_OK and wsd.status() == sa.SA_OK
+    # e2e: the query in and the outputs out every step, through pinned host buffers
+    q_host = torch.empty(q.shape, dtype=torch.int16).pin_memory()
+    q_host.copy_(q.cpu())
+    o_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    l_host = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, args.steps // 2)
+    with torch.cuda.stream(stream):
+        for it in range(e2e_steps + 2):
+            if it == 2:
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            q.copy_(q_host, non_blocking=True)
+            graph.replay()
+            o_host.copy_(out, non_blocking=True)
+            l_host.copy_(lse, non_blocking=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
+    if rank != 0:
+        return 0
+    units = g.B * g.Hq
+    achieved = pbytes / (prune_ms * 1e-3) / 1e9
+    cpu_v = cpu_done = cpu_t = None
+    if world == 1:
+        cpu_v, cpu_done, cpu_t = oracle_prune_sample(pc, args.cpu_seconds)
+    line = {
+        "metric": "sparse-decode seq*heads/s", "value": whole_job_rate(units, world, ms_per_step),
+        "unit": "seq*heads/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": "prune", "sessions": g.B, "q_heads": g.Hq, "kv_heads": g.Hkv,
+            "head_dim": g.Dk, "page": g.P, "kept_tokens": kept,
+            "tokens_before": int(d.seq_lens.sum()), "budget_tokens": d.budget,
+            "step": "sa_prune_compact of every session + one sa_sparse_decode over the "
+                    "compacted cache",
+            "l2": "inputs larger than L2: %.2f GB of K/V pool" % (
+                (k.numel() + v.numel()) * 2 / 1e9),
+            "prune_us_alone": prune_ms * 1e3, "decode_us_alone": dec_ms * 1e3,
+            "prune_algorithmic_bytes": pbytes,
+        },
+        "roofline": {"kernel": "sa_prune_compact (count, plan, position, copy kernels)",
+                     "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind + " (burst copy)",
+                     "bytes_per_launch": pbytes, "traffic": None},
+        "cpu_baseline": None if cpu_v is None else {
+            "value": cpu_v, "unit": "sessions compacted/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d sessions compacted by the oracle, %.1f s single-threaded" % (
+                cpu_done, g.B, cpu_t)},
+        "e2e": {"value": whole_job_rate(units, world, e2e_ms), "unit": "seq*heads/s",
+                "h2d_bytes_per_step": int(q.numel()) * 2,
+                "d2h_bytes_per_step": int(out.numel() + lse.numel()) * 4},
+        "gpu_launches": 8 * args.steps,  # prune: 4 kernels; decode: 4 kernels
+        "clocks": clk,
+    }
+    print(json.dumps(line, default=_json_default), flush=True)
+    return 0
+
+
 def recorded_traffic(kernel, workload):
     """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
     there is none for this workload or the kernel's source changed since it was taken."""
@@ -530,6 +731,8 @@ def main():
     try:
         if args.impl == "reference":
             rc = run_reference(args, rank, world)
+        elif args.workload == "prune":
+            rc = run_prune(args, rank, world, dist)
         else:
             rc = run_native(args, rank, world, dist)
     finally:
