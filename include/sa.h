@@ -50,7 +50,8 @@
  *      out         [B][Hq][Dv]            fp32   lse [B][Hq] fp32 (natural log)
  *  - Supported geometries: grouped-query (v_aliases_k = 0): Dk = Dv in {64, 128},
  *    G = Hq/Hkv in 1..8, Hkv <= 32; latent (v_aliases_k = 1): Hkv = 1, Dk = 576,
- *    Dv = 512, Hq = 128.  P in {16, 32, 64}.  budget, sink, window are token counts,
+ *    Dv = 512, Hq = 128 (its scores and attention are dense contractions and run on
+ *    the tcgen05 tensor cores).  P in {16, 32, 64}.  budget, sink, window are token counts,
  *    multiples of P, with sink + window <= budget.  Preconditions not checked on the
  *    device: no NaN/Inf in valid K, V, q; page_table entries of valid pages lie in
  *    [0, n_pool).
@@ -134,9 +135,11 @@ int sa_update_summaries(const sa_geom* g, const void* k_cache, const int32_t* pa
  * sum_c max(q[b][h*G+g][c] * kmax_c, q[b][h*G+g][c] * kmin_c) for p < n_b, with
  * (kmin, kmax) = summ[page_table[b][p]][h]; -inf for n_b <= p < max_pages.  fp32,
  * summation order unspecified.  q: [B][Hq][Dk] bf16, 16-byte aligned; summ as written
- * by sa_page_summaries; scores: [B][Hkv][max_pages] fp32, caller-owned.  ws: any
- * workspace of at least 256 bytes (only its status word is used: page-table entries
- * outside [0, n_pool) set SA_ERR_DEVICE_CHECK there and score as 0).  Asynchronous on
+ * by sa_page_summaries; scores: [B][Hkv][max_pages] fp32, caller-owned.  ws: for the
+ * grouped-query geometries any workspace of at least 256 bytes (only its status word is
+ * used: page-table entries outside [0, n_pool) set SA_ERR_DEVICE_CHECK there and score
+ * as 0); for the latent geometry at least sa_decode_workspace_size(g, any budget) bytes
+ * (it also holds the sign-split query rows the tensor cores read).  Asynchronous on
  * `stream`; argument errors are returned before any launch.
  * ------------------------------------------------------------------------------ */
 int sa_page_scores(const sa_geom* g, const void* q, const void* summ,
