@@ -56,6 +56,8 @@ def parse():
                     help="layer pools per step (default 32 for llama32k, 8 otherwise)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--seed", type=int, default=0,
+                    help="offset added to the workload's seed (every rank adds its own)")
     return ap.parse_args()
 
 
@@ -77,9 +79,9 @@ def peaks():
 # algorithmic bytes (inherent to the method; workspace traffic excluded)
 # ------------------------------------------------------------------------------------
 
-def rank_seed(workload, rank):
+def rank_seed(workload, rank, offset=0):
     """Seed of rank `rank`'s batch: every rank decodes its own sequences (replicas)."""
-    return synth.WORKLOADS[workload]["seed"] + 1000 * rank
+    return synth.WORKLOADS[workload]["seed"] + offset + 1000 * rank
 
 
 def max_over_ranks(x, dist, device="cpu"):
@@ -207,7 +209,22 @@ def oracle_sample(case, seconds):
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    case = synth.decode_case(args.workload)
+    if args.workload == "prune":
+        pc = synth.prune_case("prune", seed=rank_seed("prune", 0, args.seed))
+        v, done, t = oracle_prune_sample(pc, args.cpu_seconds)
+        print(json.dumps({
+            "impl": "reference", "metric": "sessions compacted/s", "value": v,
+            "unit": "sessions compacted/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "ms_per_step": None,
+            "config": {"workload": "prune"},
+            "cpu_baseline": {"value": v, "unit": "sessions compacted/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": "%d sessions compacted, %.1f s" % (done, t)},
+            "e2e": {"value": v, "unit": "sessions compacted/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}, default=_json_default), flush=True)
+        return 0
+    case = synth.decode_case(args.workload, seed=rank_seed(args.workload, 0, args.seed))
     v, done, t = oracle_sample(case, args.cpu_seconds)
     line = {
         "impl": "reference", "metric": "sparse-decode seq*heads/s", "value": v,
@@ -242,7 +259,7 @@ def run_native(args, rank, world, dist):
 
     # ---- inputs: layer 0 from the seeded generator (rank-specific seed), other layers
     # are the same bytes rolled along the page axis (distinct memory and content)
-    case = synth.decode_case(args.workload, seed=rank_seed(args.workload, rank))
+    case = synth.decode_case(args.workload, seed=rank_seed(args.workload, rank, args.seed))
     g = Geometry.of(case.geom)
     P = g.P
     L_layers = args.layers
@@ -555,7 +572,7 @@ def run_prune(args, rank, world, dist):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     hbm_peak, _, peak_kind = peaks()
-    pc = synth.prune_case("prune", seed=rank_seed("prune", rank))
+    pc = synth.prune_case("prune", seed=rank_seed("prune", rank, args.seed))
     d = pc.decode
     g = Geometry.of(d.geom)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16

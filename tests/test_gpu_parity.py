@@ -245,6 +245,58 @@ def test_mla_decode_parity(kw):
     full_parity(case, res)
 
 
+def test_mla_deterministic_bitwise():
+    case = synth.decode_case("mla", B=2, seq_lens=[30000, 9000], seed=96)
+    dc = DevCase(case)
+    a = run_decode(dc)
+    b = run_decode(dc)
+    for k in ("summ", "sel", "cnt", "out", "lse", "scores"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_sparse_decode_in_cuda_graph_replays():
+    # captured once, replayed on new queries: the outputs follow the queries exactly
+    case = synth.decode_case("llama32k", B=2, L=(8192, 8192), seed=97)
+    dc = DevCase(case)
+    g = dc.g
+    sa.page_summaries(g, dc.k, dc.pt, dc.sl, dc.summ)
+    ws = sa.Workspace.for_decode(g, case.budget)
+    out = torch.empty((g.B, g.Hq, g.Dv), dtype=torch.float32, device="cuda")
+    lse = torch.empty((g.B, g.Hq), dtype=torch.float32, device="cuda")
+    q = dc.q.clone()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        sa.sparse_decode(g, q, dc.k, dc.v, dc.summ, dc.pt, dc.sl, case.budget, case.sink,
+                         case.window, case.scale, ws, out=out, lse=lse, stream=stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            sa.sparse_decode(g, q, dc.k, dc.v, dc.summ, dc.pt, dc.sl, case.budget, case.sink,
+                             case.window, case.scale, ws, out=out, lse=lse, stream=stream)
+    rng = np.random.default_rng(97)
+    for _ in range(2):
+        qn = synth.f32_to_bf16(rng.standard_normal(case.q.shape).astype(np.float32))
+        q.copy_(to_dev(qn))
+        with torch.cuda.stream(stream):
+            graph.replay()
+        torch.cuda.synchronize()
+        assert ws.status() == sa.SA_OK
+        c2 = dataclasses.replace(case, q=qn)
+        res = dict(summ=u16(dc.summ), out=out.cpu().numpy(), lse=lse.cpu().numpy())
+        ref_out, ref_lse = sa.sparse_decode(g, q, dc.k, dc.v, dc.summ, dc.pt, dc.sl, case.budget,
+                                            case.sink, case.window, case.scale, ws)
+        assert np.array_equal(res["out"], ref_out.cpu().numpy())
+        assert np.array_equal(res["lse"], ref_lse.cpu().numpy())
+        sc = oracle.page_scores(c2.geom, c2.q, oracle.page_summaries(c2.geom, c2.k_cache,
+                                                                     c2.page_table, c2.seq_lens),
+                                c2.page_table, c2.seq_lens)
+        osel, ocnt = oracle.select_pages(c2.geom, sc, c2.seq_lens, c2.budget, c2.sink, c2.window)
+        o, l = oracle.attend(c2.geom, c2.q, c2.k_cache, c2.v_cache, c2.page_table, c2.seq_lens,
+                             osel, ocnt, c2.scale)
+        check_attention(res["out"], res["lse"], o, l)
+
+
 def test_mla_budget_covers_all_pages_equals_dense():
     case = synth.decode_case("mla", B=2, seq_lens=[1500, 777], budget=1536, seed=95)
     res = run_decode(DevCase(case))
