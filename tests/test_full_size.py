@@ -1,11 +1,18 @@
-"""Parity at the full benchmark sizes, in the launch configuration bench.py times.
+"""Parity at the full benchmark sizes.
 
-Per layer, bench.py calls select_pages (newest page's summary refreshed, physical pages of
-the selection returned) and then attend_selected with those physical pages.  Here the same
-two calls run once on the full Llama-3.1-8B-geometry workloads (batch 8, 32/8 heads,
-head dim 128, 32K or 128K tokens per sequence) and every output is compared with the
-oracle: summaries bit-exact, selection bit-exact outside the tie band, attention within
-the stated tolerance.
+bench.py decodes every layer with sa_sparse_decode, whose two halves are sa_select_pages
+(newest page's summary refreshed, physical pages of the selection returned) and
+sa_attend_selected over those physical pages: the same kernels in the same launch
+configuration.  Here the two halves run once on the full workloads and every output is
+compared with the oracle:
+- summaries bit-exact;
+- selection bit-exact outside the tie band;
+- attention within the stated tolerance.
+
+The workloads are:
+- Llama-3.1-8B geometry, batch 8, 32/8 heads, head dim 128, at 32K and 128K tokens;
+- the ragged long-context batch: 4 sequences of 64K-256K tokens, page 32;
+- the latent geometry: 16 x 64K tokens, 128 heads on one 576-wide latent.
 """
 
 import numpy as np
@@ -18,7 +25,7 @@ from parity import DevCase, check_attention, check_selection, u16
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("wl", ["llama32k", "llama128k", "mla"])
+@pytest.mark.parametrize("wl", ["llama32k", "llama128k", "ragged", "mla"])
 def test_full_size_bench_launch_config(wl):
     import torch
     import paged_kv_cache_sa_b200 as sa
@@ -62,3 +69,13 @@ def test_full_size_bench_launch_config(wl):
     o, l = oracle.attend(case.geom, case.q, case.k_cache, case.v_cache, case.page_table,
                          case.seq_lens, gs if tied else osel, ocnt, case.scale)
     check_attention(out.cpu().numpy(), lse.cpu().numpy(), o, l)
+    # the bench's own call: the same selection and bitwise the same outputs
+    sel2 = torch.empty_like(sel)
+    cnt2 = torch.empty_like(cnt)
+    out2, lse2 = sa.sparse_decode(g, dc.q, dc.k, dc.v, dc.summ, dc.pt, dc.sl, case.budget,
+                                  case.sink, case.window, case.scale, ws, sel_out=sel2,
+                                  sel_count_out=cnt2, n_tail_refresh=1)
+    assert ws.status() == sa.SA_OK
+    assert np.array_equal(sel2.cpu().numpy(), gs) and np.array_equal(cnt2.cpu().numpy(), gc)
+    assert np.array_equal(out2.cpu().numpy(), out.cpu().numpy())
+    assert np.array_equal(lse2.cpu().numpy(), lse.cpu().numpy())
