@@ -17,6 +17,7 @@ layer gives the per-phase times behind "roofline" (events between kernels cost t
 programmatic overlap of neighbouring kernels, so that pass is slightly slower).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama32k|llama128k|ragged]
+  python bench.py --select-every 4   (cross-layer reuse: select at every 4th layer only)
   python bench.py --impl reference ...   (the CPU oracle on a bounded sample)
 
 Under torchrun (N > 1) every rank runs its own batch on its own GPU (weak scaling,
@@ -58,6 +59,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--seed", type=int, default=0,
                     help="offset added to the workload's seed (every rank adds its own)")
+    ap.add_argument("--select-every", type=int, default=1,
+                    help="cross-layer selection reuse: select pages at every R-th layer and "
+                         "attend over that selection at the R-1 layers after it (default 1: "
+                         "every layer selects its own pages)")
     return ap.parse_args()
 
 
@@ -182,22 +187,28 @@ class ClockSampler:
 # CPU oracle arm (cpu_baseline and --impl reference)
 # ------------------------------------------------------------------------------------
 
-def oracle_sample(case, seconds):
+def oracle_sample(case, seconds, select_every=1):
     """Time the CPU oracle's decode step (score + select + attend) sequence by sequence
-    on the bench's own layer-0 data until ~`seconds` have elapsed."""
+    on the bench's own layer-0 data until ~`seconds` have elapsed.  With select_every=R
+    the (sequence, layer) call of layer l scores and selects only when l % R == 0 and
+    otherwise attends over the sequence's last selection."""
     import oracle
     g = case.geom
     summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
     done, t_total = 0, 0.0
     b = 0
+    last = {}
     while t_total < seconds:
         sub = synth.Geometry(1, g.Hq, g.Hkv, g.Dk, g.Dv, g.P, g.max_pages, g.n_pool, g.v_aliases_k)
         q = case.q[b:b + 1]
         pt = case.page_table[b:b + 1]
         sl = case.seq_lens[b:b + 1]
+        layer = done // g.B
         t0 = time.perf_counter()
-        sc = oracle.page_scores(sub, q, summ, pt, sl)
-        sel, cnt = oracle.select_pages(sub, sc, sl, case.budget, case.sink, case.window)
+        if layer % select_every == 0 or b not in last:
+            sc = oracle.page_scores(sub, q, summ, pt, sl)
+            last[b] = oracle.select_pages(sub, sc, sl, case.budget, case.sink, case.window)
+        sel, cnt = last[b]
         oracle.attend(sub, q, case.k_cache, case.v_cache, pt, sl, sel, cnt, case.scale)
         t_total += time.perf_counter() - t0
         done += 1
@@ -225,17 +236,20 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}, default=_json_default), flush=True)
         return 0
     case = synth.decode_case(args.workload, seed=rank_seed(args.workload, 0, args.seed))
-    v, done, t = oracle_sample(case, args.cpu_seconds)
+    v, done, t = oracle_sample(case, args.cpu_seconds, args.select_every)
     line = {
         "impl": "reference", "metric": "sparse-decode seq*heads/s", "value": v,
         "unit": "seq*heads/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "ms_per_step": None,
-        "config": {"workload": args.workload, "layers_per_step": args.layers},
+        "config": {"workload": args.workload, "layers_per_step": args.layers,
+                   "select_every": args.select_every},
         "cpu_baseline": {"value": v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
                          "sample": "%d (sequence, layer) decode calls of layer 0 "
-                                   "(score+select+attend, all %d heads), %.1f s" % (
-                                       done, case.geom.Hq, t)},
+                                   "(score+select%s, attend; all %d heads), %.1f s" % (
+                                       done, "" if args.select_every == 1 else
+                                       " every %d layers" % args.select_every,
+                                       case.geom.Hq, t)},
         "e2e": {"value": v, "unit": "seq*heads/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -303,12 +317,26 @@ def run_native(args, rank, world, dist):
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
           for _ in range(L_layers)]
 
+    R = args.select_every
+
     def step_fused():
         # the headline: one sa_sparse_decode per layer (selection + attention)
+        if R == 1:
+            for l in range(L_layers):
+                sa.sparse_decode(g, qs[l], ks[l], vs[l], summs[l], pt, sl, case.budget,
+                                 case.sink, case.window, case.scale, ws, out=outs[l],
+                                 lse=lses[l], sel_out=sel, sel_count_out=cnt, n_tail_refresh=1)
+            return
+        # cross-layer reuse: layer l selects when l % R == 0; the layers after it attend
+        # over that selection (physical pages of the shared page table) with their own
+        # query, keys and values
         for l in range(L_layers):
-            sa.sparse_decode(g, qs[l], ks[l], vs[l], summs[l], pt, sl, case.budget, case.sink,
-                             case.window, case.scale, ws, out=outs[l], lse=lses[l],
-                             sel_out=sel, sel_count_out=cnt, n_tail_refresh=1)
+            if l % R == 0:
+                sa.select_pages(g, qs[l], summs[l], pt, sl, case.budget, case.sink,
+                                case.window, ws, sel=sel, sel_count=cnt, k_cache=ks[l],
+                                n_tail_refresh=1, sel_phys=phys)
+            sa.attend_selected(g, qs[l], ks[l], vs[l], pt, sl, sel, cnt, case.scale, ws,
+                               out=outs[l], lse=lses[l], sel_phys=phys)
 
     def step(with_events):
         for l in range(L_layers):
@@ -329,7 +357,8 @@ def run_native(args, rank, world, dist):
     assert ws.status() == sa.SA_OK
     sel_count = cnt.cpu().numpy()
     sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, P)
-    step_bytes = L_layers * (sel_b + att_b + upd_b)
+    n_sel_layers = (L_layers + R - 1) // R
+    step_bytes = L_layers * att_b + n_sel_layers * (sel_b + upd_b)
 
     # the dominant kernel alone (page scoring of every layer), an event pair per launch
     ev_sc = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
@@ -445,10 +474,12 @@ def run_native(args, rank, world, dist):
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     cpu_v, cpu_done, cpu_t = (None, 0, 0.0)
     if world == 1:
-        cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds)
+        cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds, R)
     # GQA: score, select (+ tail refresh), attention, merge; latent: tail refresh, query
     # sign split, tensor-core score, select, tensor-core attention, merge
-    launches_per_layer = 6 if g.v_aliases_k else 4
+    launches_select = 4 if g.v_aliases_k else 2   # select half of one layer-call
+    launches_attend = 2                           # attention + merge
+    launches_per_step = n_sel_layers * launches_select + L_layers * launches_attend
     line = {
         "metric": "sparse-decode seq*heads/s",
         "value": value,
@@ -467,6 +498,8 @@ def run_native(args, rank, world, dist):
             "batch": g.B, "q_heads": g.Hq, "kv_heads": g.Hkv, "head_dim": g.Dk,
             "seq_len": int(case.seq_lens.max()), "page": P, "budget_tokens": case.budget,
             "sink": case.sink, "window": case.window, "layers_per_step": L_layers,
+            "select_every": R,
+            "call": "sa_sparse_decode" if R == 1 else "sa_select_pages + sa_attend_selected",
             "l2": "inputs larger than L2: %d distinct layer pools, %.2f GB touched per step"
                   % (L_layers, step_bytes / 1e9),
             "parallelism": "replicas (batch split), no collective" if world > 1 else "1 GPU",
@@ -478,7 +511,7 @@ def run_native(args, rank, world, dist):
             "page_scores_us_alone": sc_mean * 1e3,
             "summaries_us_alone": summ_ms * 1e3,
             "summaries_gbs_alone": summ_bytes / (summ_ms * 1e-3) / 1e9,
-            "algorithmic_bytes_per_layer": sel_b + att_b + upd_b,
+            "algorithmic_bytes_per_layer": step_bytes / L_layers,
             **mla_flops(case, sel_count, sc_mean, att_mean),
         },
         "roofline": {
@@ -490,11 +523,12 @@ def run_native(args, rank, world, dist):
         },
         "cpu_baseline": None if cpu_v is None else {
             "value": cpu_v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
-            "sample": "%d (sequence, layer) decode calls of layer 0 (score+select+attend over "
-                      "all %d query heads), %.1f s single-threaded" % (cpu_done, g.Hq, cpu_t)},
+            "sample": "%d (sequence, layer) decode calls of layer 0 (score+select%s, attend; "
+                      "all %d query heads), %.1f s single-threaded" % (
+                          cpu_done, "" if R == 1 else " every %d layers" % R, g.Hq, cpu_t)},
         "e2e": {"value": whole_job_rate(units_per_step, world, e2e_ms), "unit": "seq*heads/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_layer * L_layers * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
     print(json.dumps(line, default=_json_default), flush=True)
@@ -730,6 +764,8 @@ def recorded_traffic(kernel, workload):
 
 def main():
     args = parse()
+    if args.select_every < 1:
+        raise SystemExit("--select-every must be >= 1")
     if args.layers is None:
         args.layers = N_LAYERS if args.workload == "llama32k" else 8
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -7,7 +7,8 @@ import pytest
 
 import oracle
 import synth
-from parity import DevCase, check_attention, full_parity, run_decode, to_dev, u16
+from parity import (DevCase, check_attention, check_selection, full_parity, run_decode, to_dev,
+                    u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -348,6 +349,42 @@ def test_attend_selected_reuses_indices():
     ro, rl = oracle.attend(c2.geom, c2.q, c2.k_cache, c2.v_cache, c2.page_table, c2.seq_lens,
                            r1["sel"], r1["cnt"], c2.scale)
     check_attention(out.cpu().numpy(), lse.cpu().numpy(), ro, rl)
+
+
+def test_cross_layer_reuse_of_physical_pages():
+    # layer 0 selects and returns the physical pages of its selection; the next layer
+    # (own q, K, V; the same page table and lengths) attends over those physical pages
+    lens = [4096, 1000, 2500]
+    c0 = synth.decode_case("llama32k", B=3, seq_lens=lens, seed=41)
+    other = synth.decode_case("llama32k", B=3, seq_lens=lens, seed=42)
+    assert other.k_cache.shape == c0.k_cache.shape
+    c1 = dataclasses.replace(c0, q=other.q, k_cache=other.k_cache, v_cache=other.v_cache)
+    d0, d1 = DevCase(c0), DevCase(c1)
+    g = d0.g
+    K = c0.budget // g.P
+    ws = sa.Workspace.for_decode(g, c0.budget)
+    sa.page_summaries(g, d0.k, d0.pt, d0.sl, d0.summ)
+    sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((g.B, g.Hkv), dtype=torch.int32, device="cuda")
+    phys = torch.empty_like(sel)
+    sa.select_pages(g, d0.q, d0.summ, d0.pt, d0.sl, c0.budget, c0.sink, c0.window, ws,
+                    sel=sel, sel_count=cnt, sel_phys=phys)
+    out, lse = sa.attend_selected(g, d1.q, d1.k, d1.v, d1.pt, d1.sl, sel, cnt, c1.scale, ws,
+                                  sel_phys=phys)
+    assert ws.status() == sa.SA_OK
+    gs, gc = sel.cpu().numpy(), cnt.cpu().numpy()
+    summ = oracle.page_summaries(c0.geom, c0.k_cache, c0.page_table, c0.seq_lens)
+    sc = oracle.page_scores(c0.geom, c0.q, summ, c0.page_table, c0.seq_lens)
+    osel, ocnt = oracle.select_pages(c0.geom, sc, c0.seq_lens, c0.budget, c0.sink, c0.window)
+    tied = check_selection(c0.geom, c0.seq_lens, c0.budget, c0.sink, c0.window, sc, osel, ocnt,
+                           gs, gc)
+    ro, rl = oracle.attend(c1.geom, c1.q, c1.k_cache, c1.v_cache, c1.page_table, c1.seq_lens,
+                           gs if tied else osel, ocnt, c1.scale)
+    check_attention(out.cpu().numpy(), lse.cpu().numpy(), ro, rl)
+    # the same outputs as when layer 1 looks its pages up through the page table itself
+    out2, lse2 = sa.attend_selected(g, d1.q, d1.k, d1.v, d1.pt, d1.sl, sel, cnt, c1.scale, ws)
+    assert np.array_equal(out2.cpu().numpy(), out.cpu().numpy())
+    assert np.array_equal(lse2.cpu().numpy(), lse.cpu().numpy())
 
 
 def test_deterministic_bitwise():
