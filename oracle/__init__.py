@@ -24,7 +24,8 @@ _SRC = os.path.join(_HERE, "sa_oracle.c")
 _LIB = os.path.join(_HERE, "lib", "libsa_oracle.so")
 
 __all__ = ["build", "load", "page_summaries", "page_scores", "select_pages", "attend",
-           "dense_attend", "prune_compact", "decode"]
+           "dense_attend", "prune_compact", "decode", "e4m3_values", "e4m3_outward",
+           "page_summaries_fp8", "page_scores_fp8", "decode_fp8"]
 
 
 class _Geom(ctypes.Structure):
@@ -67,6 +68,14 @@ def load():
         lib.oracle_prune_compact.argtypes = [ctypes.POINTER(_Geom), P, P, P, P, P, P,
                                              ctypes.c_int64, P, P, P, P, P, P, P]
         lib.oracle_prune_compact.restype = ctypes.c_int64
+        lib.oracle_e4m3_values.argtypes = [P]
+        lib.oracle_e4m3_values.restype = None
+        lib.oracle_e4m3_outward.argtypes = [ctypes.c_double, i32]
+        lib.oracle_e4m3_outward.restype = ctypes.c_uint8
+        lib.oracle_encode_fp8.argtypes = [ctypes.POINTER(_Geom), P, P, P, P]
+        lib.oracle_encode_fp8.restype = None
+        lib.oracle_page_scores_fp8.argtypes = [ctypes.POINTER(_Geom), P, P, P, P, P]
+        lib.oracle_page_scores_fp8.restype = None
         _lib = lib
     return _lib
 
@@ -101,6 +110,40 @@ def page_scores(geom, q, summ, page_table, seq_lens) -> np.ndarray:
     out = np.empty((geom.B, geom.Hkv, geom.max_pages), dtype=np.float64)
     g = _geom(geom)
     load().oracle_page_scores(ctypes.byref(g), _p(q), _p(summ), _p(pt), _p(sl), _p(out))
+    return out
+
+
+def e4m3_values() -> np.ndarray:
+    """Value of each of the 256 FP8 E4M3 codes (NaN for 0x7F and 0xFF)."""
+    out = np.empty(256, dtype=np.float64)
+    load().oracle_e4m3_values(_p(out))
+    return out
+
+
+def e4m3_outward(x: float, up: bool) -> int:
+    """Tightest finite E4M3 code >= x (up) or <= x (down); zero is 0x00."""
+    return int(load().oracle_e4m3_outward(float(x), 1 if up else 0))
+
+
+def page_summaries_fp8(geom, k_cache, page_table, seq_lens) -> np.ndarray:
+    """fp8 records [n_pool, Hkv, 2*Dk + 16] uint8 of every used page: Dk codes of the
+    min row (rounded toward -inf), Dk codes of the max row (toward +inf), the int8
+    exponent e, 15 zero bytes; values = code * 2^e.  Untouched pages are 0."""
+    summ = page_summaries(geom, k_cache, page_table, seq_lens)
+    out = np.zeros((geom.n_pool, geom.Hkv, 2 * geom.Dk + 16), dtype=np.uint8)
+    pt, sl = _c(page_table, np.int32), _c(seq_lens, np.int32)
+    g = _geom(geom)
+    load().oracle_encode_fp8(ctypes.byref(g), _p(summ), _p(pt), _p(sl), _p(out))
+    return out
+
+
+def page_scores_fp8(geom, q, summ8, page_table, seq_lens) -> np.ndarray:
+    """The page bound over decoded fp8 records: [B, Hkv, max_pages] float64."""
+    q, summ8 = _c(q, np.uint16), _c(summ8, np.uint8)
+    pt, sl = _c(page_table, np.int32), _c(seq_lens, np.int32)
+    out = np.empty((geom.B, geom.Hkv, geom.max_pages), dtype=np.float64)
+    g = _geom(geom)
+    load().oracle_page_scores_fp8(ctypes.byref(g), _p(q), _p(summ8), _p(pt), _p(sl), _p(out))
     return out
 
 
@@ -190,4 +233,19 @@ def decode(case, sel=None, sel_count=None):
     out, lse = attend(g, case.q, case.k_cache, case.v_cache, case.page_table, case.seq_lens,
                       sel, sel_count, case.scale)
     return dict(summ=summ, scores=scores, sel=osel, sel_count=ocnt, out=out, lse=lse,
+                attend_sel=sel, attend_count=sel_count)
+
+
+def decode_fp8(case, sel=None, sel_count=None):
+    """``decode`` with the page bound taken over fp8 summaries rounded outward
+    (page_summaries_fp8 / page_scores_fp8); attention still reads the bf16 K and V."""
+    g = case.geom
+    summ8 = page_summaries_fp8(g, case.k_cache, case.page_table, case.seq_lens)
+    scores = page_scores_fp8(g, case.q, summ8, case.page_table, case.seq_lens)
+    osel, ocnt = select_pages(g, scores, case.seq_lens, case.budget, case.sink, case.window)
+    if sel is None:
+        sel, sel_count = osel, ocnt
+    out, lse = attend(g, case.q, case.k_cache, case.v_cache, case.page_table, case.seq_lens,
+                      sel, sel_count, case.scale)
+    return dict(summ8=summ8, scores=scores, sel=osel, sel_count=ocnt, out=out, lse=lse,
                 attend_sel=sel, attend_count=sel_count)

@@ -140,6 +140,124 @@ ORACLE_API void oracle_page_scores(const oracle_geom* g, const uint16_t* q,
     }
 }
 
+/* (2') fp8 summaries rounded outward, and the page bound over them.  The SparseEngine
+ * blog's hook-point paragraph lists quantised KV (KIVI) next to Quest; the pages give
+ * no format.  Reading taken: OCP FP8 E4M3 ("fn": bias 7, no infinities, 0x7F/0xFF
+ * NaN) codes of the min row rounded toward -inf and of the max row rounded toward
+ * +inf, after scaling the (page, KV head) record by 2^-e, e the smallest integer with
+ * max|value| * 2^-e <= 448 (the largest finite code).  The decoded record then still
+ * brackets every key of the page, so the bound stays an upper bound.
+ * Record: [Dk codes of min][Dk codes of max][int8 e][15 zero bytes]. */
+
+/* Value of an E4M3 code from the format's definition. */
+static double e4m3_value(int code) {
+    int s = (code >> 7) & 1, E = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (E == 15 && m == 7) return NAN;
+    if (E == 0)
+        v = ldexp((double)m, -9);          /* subnormal: (m/8) * 2^(1-7) */
+    else
+        v = ldexp(1.0 + m / 8.0, E - 7);
+    return s ? -v : v;
+}
+
+ORACLE_API void oracle_e4m3_values(double* out) {
+    for (int c = 0; c < 256; ++c) out[c] = e4m3_value(c);
+}
+
+/* The tightest finite code >= x (up) or <= x (down), found by trying all of them; a
+ * zero result is the code 0x00.  0x7F (NaN) when no finite code qualifies. */
+static uint8_t e4m3_outward(double x, int up) {
+    int best = -1;
+    double bv = 0.0;
+    for (int c = 0; c < 256; ++c) {
+        double v = e4m3_value(c);
+        if (isnan(v)) continue;
+        if (up ? !(v >= x) : !(v <= x)) continue;
+        if (best < 0 || (up ? v < bv : v > bv)) {
+            best = c;
+            bv = v;
+        }
+    }
+    if (best < 0) return 0x7F;
+    return bv == 0.0 ? 0x00 : (uint8_t)best;
+}
+
+ORACLE_API uint8_t oracle_e4m3_outward(double x, int up) { return e4m3_outward(x, up); }
+
+/* smallest integer e with A * 2^-e <= 448; 0 when A == 0 */
+static int fp8_exponent(double A) {
+    if (A == 0.0) return 0;
+    int e = -400;
+    while (ldexp(A, -e) > 448.0) ++e;
+    return e;
+}
+
+/* Encode the bf16 summaries of every page a sequence uses into fp8 records. */
+ORACLE_API void oracle_encode_fp8(const oracle_geom* g, const uint16_t* summ,
+                                  const int32_t* page_table, const int32_t* seq_lens,
+                                  uint8_t* summ8) {
+    const int64_t rec = 2 * (int64_t)g->Dk + 16;
+    for (int b = 0; b < g->B; ++b) {
+        int64_t nb = n_pages_of(seq_lens[b], g->P);
+        for (int64_t lp = 0; lp < nb; ++lp) {
+            int64_t phys = page_table[(int64_t)b * g->max_pages + lp];
+            for (int h = 0; h < g->Hkv; ++h) {
+                const uint16_t* kmin = summ + ((phys * g->Hkv + h) * 2) * (int64_t)g->Dk;
+                const uint16_t* kmax = kmin + g->Dk;
+                uint8_t* out = summ8 + (phys * g->Hkv + h) * rec;
+                double A = 0.0;
+                for (int c = 0; c < g->Dk; ++c) {
+                    if (fabs(bf(kmin[c])) > A) A = fabs(bf(kmin[c]));
+                    if (fabs(bf(kmax[c])) > A) A = fabs(bf(kmax[c]));
+                }
+                int e = fp8_exponent(A);
+                for (int c = 0; c < g->Dk; ++c) {
+                    out[c] = e4m3_outward(ldexp(bf(kmin[c]), -e), 0);
+                    out[g->Dk + c] = e4m3_outward(ldexp(bf(kmax[c]), -e), 1);
+                }
+                memset(out + 2 * g->Dk, 0, 16);
+                out[2 * g->Dk] = (uint8_t)(int8_t)e;
+            }
+        }
+    }
+}
+
+/* The page bound of (2) over decoded fp8 records: kmin_c = value(code) * 2^e, the same
+ * for kmax; in double (exact: a bf16 times a 4-bit-significand value scaled by 2^e). */
+ORACLE_API void oracle_page_scores_fp8(const oracle_geom* g, const uint16_t* q,
+                                       const uint8_t* summ8, const int32_t* page_table,
+                                       const int32_t* seq_lens, double* scores) {
+    int G = g->Hq / g->Hkv;
+    const int64_t rec = 2 * (int64_t)g->Dk + 16;
+    for (int b = 0; b < g->B; ++b) {
+        int64_t nb = n_pages_of(seq_lens[b], g->P);
+        for (int h = 0; h < g->Hkv; ++h) {
+            double* srow = scores + ((int64_t)b * g->Hkv + h) * g->max_pages;
+            for (int64_t lp = 0; lp < g->max_pages; ++lp) {
+                if (lp >= nb) { srow[lp] = -INFINITY; continue; }
+                int64_t phys = page_table[(int64_t)b * g->max_pages + lp];
+                const uint8_t* r = summ8 + (phys * g->Hkv + h) * rec;
+                int e = (int8_t)r[2 * g->Dk];
+                double best = -INFINITY;
+                for (int gi = 0; gi < G; ++gi) {
+                    const uint16_t* qg = q + ((int64_t)b * g->Hq + h * G + gi) * g->Dk;
+                    double u = 0.0;
+                    for (int c = 0; c < g->Dk; ++c) {
+                        double lo = ldexp(e4m3_value(r[c]), e);
+                        double hi = ldexp(e4m3_value(r[g->Dk + c]), e);
+                        double a = bf(qg[c]) * hi;
+                        double d = bf(qg[c]) * lo;
+                        u += (a > d) ? a : d;
+                    }
+                    if (u > best) best = u;
+                }
+                srow[lp] = best;
+            }
+        }
+    }
+}
+
 typedef struct { double s; int32_t p; } cand;
 
 /* higher score first; equal scores -> lower logical page index first */

@@ -474,3 +474,113 @@ def test_decode_after_prune_full_budget_equals_dense_on_kept_tokens():
                                          d.scale)
             assert np.allclose(out[b, h * g.G:(h + 1) * g.G], od, rtol=0, atol=1e-12)
             assert np.allclose(lse[b, h * g.G:(h + 1) * g.G], ld, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------
+# fp8 summaries rounded outward (E4M3 codes, one power-of-two exponent per record)
+# ------------------------------------------------------------------------------------
+
+def test_e4m3_table_matches_torch_float8():
+    # the library routine: torch's float8_e4m3fn decoding of all 256 bytes
+    import torch
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    v = oracle.e4m3_values()
+    assert np.array_equal(np.isnan(v), np.isnan(ref))
+    assert np.array_equal(v[~np.isnan(v)], ref[~np.isnan(ref)].astype(np.float64))
+    assert v[0x7E] == 448.0 and v[0x01] == 2.0 ** -9 and v[0x08] == 2.0 ** -6
+
+
+def test_e4m3_outward_is_the_tightest_bracket_and_brackets_torch_rounding():
+    import torch
+    v = oracle.e4m3_values()
+    fin = np.sort(np.unique(v[~np.isnan(v)]))
+    rng = np.random.default_rng(8)
+    xs = np.concatenate([rng.uniform(-448, 448, 300), rng.standard_normal(300) * 0.01,
+                         fin, [0.0, -0.0, 448.0, -448.0, 2.0 ** -10, -(2.0 ** -10)]])
+    xs = xs.astype(np.float32).astype(np.float64)
+    rne = torch.from_numpy(xs.astype(np.float32)).to(torch.float8_e4m3fn).float().numpy()
+    for x, r in zip(xs, rne):
+        dn, up = v[oracle.e4m3_outward(x, False)], v[oracle.e4m3_outward(x, True)]
+        assert dn <= x <= up
+        # nothing representable strictly inside (dn, x) or (x, up)
+        assert not np.any((fin > dn) & (fin < x)) and not np.any((fin > x) & (fin < up))
+        assert r in (dn, up)                    # round-to-nearest picks one of the two
+        if x in fin:
+            assert dn == up == x
+    assert oracle.e4m3_outward(0.0, True) == 0 and oracle.e4m3_outward(-0.0, False) == 0
+    assert oracle.e4m3_outward(-(2.0 ** -12), True) == 0          # toward +inf: zero
+    assert oracle.e4m3_outward(2.0 ** -12, True) == 0x01          # up: smallest subnormal
+
+
+def test_fp8_worked_record():
+    # one page, one head, Dk = 64: channel 0 holds -1.1 and 3.3 (bf16 -1.1015625 and
+    # 3.296875), every other channel 0.  A = 3.296875: 3.296875 * 2^7 = 422 <= 448 and
+    # 3.296875 * 2^8 > 448, so e = -7.  max row: 422 lies in [256, 512), step 32 ->
+    # up to 448 = code 0x7E.  min row: -1.1015625 * 128 = -141 lies in [-256, -128),
+    # step 16 -> down to -144 = 1.125 * 2^7 -> E = 14, m = 1 -> 0x71 | sign = 0xF1.
+    case = synth.decode_case("tiny", B=1, seq_lens=[2], Hkv=1, Hq=1, Dk=64)
+    k = np.zeros_like(case.k_cache)
+    ph = case.page_table[0, 0]
+    k[ph, 0, 0, 0] = _bf([-1.1])[0]
+    k[ph, 0, 1, 0] = _bf([3.3])[0]
+    case = dataclasses.replace(case, k_cache=k)
+    r = oracle.page_summaries_fp8(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    rec = r[ph, 0]
+    assert rec.shape == (2 * 64 + 16,)
+    assert rec[0] == 0xF1 and rec[64] == 0x7E
+    assert (rec[1:64] == 0).all() and (rec[65:128] == 0).all()
+    assert rec[128].view(np.int8) == -7 and (rec[129:] == 0).all()
+
+
+def _decoded_fp8(case, r):
+    v = oracle.e4m3_values()
+    D = case.geom.Dk
+    e = r[..., 2 * D].view(np.int8).astype(np.float64)[..., None]
+    return v[r[..., :D]] * 2.0 ** e, v[r[..., D:2 * D]] * 2.0 ** e
+
+
+@pytest.mark.parametrize("wl,kw", [("tiny", dict(B=3, seq_lens=[4096, 700, 33], Hkv=2, Hq=8)),
+                                   ("ragged", dict(B=2, L=(3000, 5000), seed=15))])
+def test_fp8_records_bracket_the_bf16_summaries(wl, kw):
+    case = synth.decode_case(wl, **kw)
+    g = case.geom
+    s16 = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    r = oracle.page_summaries_fp8(g, case.k_cache, case.page_table, case.seq_lens)
+    used = np.unique(np.concatenate([case.page_table[b, :(case.seq_lens[b] + g.P - 1) // g.P]
+                                     for b in range(g.B)]))
+    lo, hi = _decoded_fp8(case, r[used])
+    kmin = bf16_to_f32(s16[used, :, 0]).astype(np.float64)
+    kmax = bf16_to_f32(s16[used, :, 1]).astype(np.float64)
+    assert (lo <= kmin).all() and (hi >= kmax).all()
+    # the exponent puts each record's largest magnitude into (224, 448]
+    A = np.maximum(np.abs(kmin).max(-1), np.abs(kmax).max(-1))
+    e = r[used][..., 2 * g.Dk].view(np.int8).astype(np.float64)
+    scaled = A * 2.0 ** -e
+    assert ((scaled > 224) & (scaled <= 448) | (A == 0)).all()
+    assert (r[used][..., 2 * g.Dk + 1:] == 0).all()
+    # outward by at most one step: relative widening below 2^-3 for normal codes
+    big = np.abs(kmax) * 2.0 ** -e[..., None] >= 2.0 ** -6
+    assert (np.abs(hi - kmax)[big] <= np.abs(kmax)[big] * 2.0 ** -3).all()
+
+
+def test_fp8_bound_dominates_the_bf16_bound_and_equals_it_on_representable_keys():
+    case = synth.decode_case("tiny", B=2, seq_lens=[2048, 500], Hkv=2, Hq=8, seed=9)
+    g = case.geom
+    s16 = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    sc16 = oracle.page_scores(g, case.q, s16, case.page_table, case.seq_lens)
+    r = oracle.page_summaries_fp8(g, case.k_cache, case.page_table, case.seq_lens)
+    sc8 = oracle.page_scores_fp8(g, case.q, r, case.page_table, case.seq_lens)
+    fin = np.isfinite(sc16)
+    assert np.array_equal(fin, np.isfinite(sc8))
+    assert (sc8[fin] >= sc16[fin] - 1e-9 * np.abs(sc16[fin])).all()
+    assert (sc8[fin] > sc16[fin]).any()
+    # keys drawn from values whose scaled forms are exact codes: 3 * 2^7 = 384 etc.
+    rng = np.random.default_rng(9)
+    vals = _bf([-2.0, -1.0, -0.5, 0.0, 0.5, 1.0, 3.0])
+    k = vals[rng.integers(0, len(vals), size=case.k_cache.shape)]
+    case2 = dataclasses.replace(case, k_cache=k)
+    s16 = oracle.page_summaries(g, case2.k_cache, case2.page_table, case2.seq_lens)
+    r = oracle.page_summaries_fp8(g, case2.k_cache, case2.page_table, case2.seq_lens)
+    a = oracle.page_scores(g, case2.q, s16, case2.page_table, case2.seq_lens)
+    b = oracle.page_scores_fp8(g, case2.q, r, case2.page_table, case2.seq_lens)
+    assert np.array_equal(a, b)
