@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--seed", type=int, default=0,
                     help="offset added to the workload's seed (every rank adds its own)")
+    ap.add_argument("--summaries", default="bf16", choices=["bf16", "fp8"],
+                    help="fp8: page summaries as E4M3 records rounded outward "
+                         "(sa_sparse_decode_fp8); grouped-query workloads only")
     ap.add_argument("--select-every", type=int, default=1,
                     help="cross-layer selection reuse: select pages at every R-th layer and "
                          "attend over that selection at the R-1 layers after it (default 1: "
@@ -105,11 +108,13 @@ def whole_job_rate(units_per_rank_step, world, ms_per_step):
     return units_per_rank_step * world / (ms_per_step * 1e-3)
 
 
-def layer_bytes(geom, seq_lens, sel_count, P):
-    """Per layer-call: (select_bytes, attend_bytes, update_bytes)."""
+def layer_bytes(geom, seq_lens, sel_count, P, fp8=False):
+    """Per layer-call: (select_bytes, attend_bytes, update_bytes).  fp8: summaries are
+    records of 2*Dk + 16 bytes per (page, KV head) instead of 4*Dk."""
     g = geom
+    rec = 2 * g.Dk + 16 if fp8 else 4 * g.Dk
     nb = (seq_lens.astype(np.int64) + P - 1) // P
-    summ = int(nb.sum()) * g.Hkv * 2 * g.Dk * 2
+    summ = int(nb.sum()) * g.Hkv * rec
     pt = int(nb.sum()) * 4
     q = g.B * g.Hq * g.Dk * 2
     sel_bytes = summ + pt + q
@@ -124,7 +129,7 @@ def layer_bytes(geom, seq_lens, sel_count, P):
             tok += c * P - (P - last_valid if c else 0)
     kv = tok * (g.Dk + (0 if g.v_aliases_k else g.Dv)) * 2
     att_bytes = kv + q + g.B * g.Hq * (g.Dv * 4 + 4)
-    upd = g.B * g.Hkv * (P * g.Dk * 2 + 2 * g.Dk * 2)
+    upd = g.B * g.Hkv * (P * g.Dk * 2 + rec)
     return sel_bytes, att_bytes, upd
 
 
@@ -187,14 +192,20 @@ class ClockSampler:
 # CPU oracle arm (cpu_baseline and --impl reference)
 # ------------------------------------------------------------------------------------
 
-def oracle_sample(case, seconds, select_every=1):
+def oracle_sample(case, seconds, select_every=1, fp8=False):
     """Time the CPU oracle's decode step (score + select + attend) sequence by sequence
     on the bench's own layer-0 data until ~`seconds` have elapsed.  With select_every=R
     the (sequence, layer) call of layer l scores and selects only when l % R == 0 and
-    otherwise attends over the sequence's last selection."""
+    otherwise attends over the sequence's last selection.  fp8: scores over the fp8
+    records."""
     import oracle
     g = case.geom
-    summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+    if fp8:
+        summ = oracle.page_summaries_fp8(g, case.k_cache, case.page_table, case.seq_lens)
+        scorer = oracle.page_scores_fp8
+    else:
+        summ = oracle.page_summaries(g, case.k_cache, case.page_table, case.seq_lens)
+        scorer = oracle.page_scores
     done, t_total = 0, 0.0
     b = 0
     last = {}
@@ -206,7 +217,7 @@ def oracle_sample(case, seconds, select_every=1):
         layer = done // g.B
         t0 = time.perf_counter()
         if layer % select_every == 0 or b not in last:
-            sc = oracle.page_scores(sub, q, summ, pt, sl)
+            sc = scorer(sub, q, summ, pt, sl)
             last[b] = oracle.select_pages(sub, sc, sl, case.budget, case.sink, case.window)
         sel, cnt = last[b]
         oracle.attend(sub, q, case.k_cache, case.v_cache, pt, sl, sel, cnt, case.scale)
@@ -236,14 +247,15 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}, default=_json_default), flush=True)
         return 0
     case = synth.decode_case(args.workload, seed=rank_seed(args.workload, 0, args.seed))
-    v, done, t = oracle_sample(case, args.cpu_seconds, args.select_every)
+    v, done, t = oracle_sample(case, args.cpu_seconds, args.select_every,
+                               args.summaries == "fp8")
     line = {
         "impl": "reference", "metric": "sparse-decode seq*heads/s", "value": v,
         "unit": "seq*heads/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "ms_per_step": None,
         "config": {"workload": args.workload, "layers_per_step": args.layers,
-                   "select_every": args.select_every},
+                   "select_every": args.select_every, "summaries": args.summaries},
         "cpu_baseline": {"value": v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
                          "sample": "%d (sequence, layer) decode calls of layer 0 "
                                    "(score+select%s, attend; all %d heads), %.1f s" % (
@@ -276,6 +288,9 @@ def run_native(args, rank, world, dist):
     case = synth.decode_case(args.workload, seed=rank_seed(args.workload, rank, args.seed))
     g = Geometry.of(case.geom)
     P = g.P
+    F8 = args.summaries == "fp8"
+    if F8 and (g.v_aliases_k or args.select_every != 1):
+        raise SystemExit("--summaries fp8 needs a grouped-query workload and --select-every 1")
     L_layers = args.layers
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16
                                                           else a)).to(dev)
@@ -291,20 +306,27 @@ def run_native(args, rank, world, dist):
                   (v0 if l == 0 else torch.roll(v0, shifts=l * stride, dims=0)))
         qn = case.q if l == 0 else synth.f32_to_bf16(rng.standard_normal(case.q.shape).astype(np.float32))
         qs.append(t(qn))
-        summs.append(torch.empty((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device=dev))
-        sa.page_summaries(g, ks[l], pt, sl, summs[l])
+        if F8:
+            summs.append(sa.empty_summaries_fp8(g, dev))
+            sa.page_summaries_fp8(g, ks[l], pt, sl, summs[l])
+        else:
+            summs.append(torch.empty((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device=dev))
+            sa.page_summaries(g, ks[l], pt, sl, summs[l])
     # per-page summaries (row a-1) of one layer's pool, timed alone: K read once
     e_s0, e_s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e_s0.record()
     for _ in range(3):
-        sa.page_summaries(g, ks[0], pt, sl, summs[0])
+        if F8:
+            sa.page_summaries_fp8(g, ks[0], pt, sl, summs[0])
+        else:
+            sa.page_summaries(g, ks[0], pt, sl, summs[0])
     e_s1.record()
     torch.cuda.synchronize()
     summ_ms = e_s0.elapsed_time(e_s1) / 3
     n_used = int(((case.seq_lens.astype(np.int64) + P - 1) // P).sum())
     summ_bytes = int(case.seq_lens.astype(np.int64).sum()) * g.Hkv * g.Dk * 2 + \
-        n_used * g.Hkv * 2 * g.Dk * 2 + n_used * 4
+        n_used * g.Hkv * (2 * g.Dk + 16 if F8 else 4 * g.Dk) + n_used * 4
     K = case.budget // P
     ws = sa.Workspace.for_decode(g, case.budget)
     sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device=dev)
@@ -321,6 +343,13 @@ def run_native(args, rank, world, dist):
 
     def step_fused():
         # the headline: one sa_sparse_decode per layer (selection + attention)
+        if F8:
+            for l in range(L_layers):
+                sa.sparse_decode_fp8(g, qs[l], ks[l], vs[l], summs[l], pt, sl, case.budget,
+                                     case.sink, case.window, case.scale, ws, out=outs[l],
+                                     lse=lses[l], sel_out=sel, sel_count_out=cnt,
+                                     n_tail_refresh=1)
+            return
         if R == 1:
             for l in range(L_layers):
                 sa.sparse_decode(g, qs[l], ks[l], vs[l], summs[l], pt, sl, case.budget,
@@ -356,7 +385,7 @@ def run_native(args, rank, world, dist):
     step_fused()
     assert ws.status() == sa.SA_OK
     sel_count = cnt.cpu().numpy()
-    sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, P)
+    sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, P, F8)
     n_sel_layers = (L_layers + R - 1) // R
     step_bytes = L_layers * att_b + n_sel_layers * (sel_b + upd_b)
 
@@ -368,7 +397,10 @@ def run_native(args, rank, world, dist):
     def score_only():
         for l in range(L_layers):
             ev_sc[l][0].record()
-            sa.page_scores(g, qs[l], summs[l], pt, sl, ws, scores=scores_buf)
+            if F8:
+                sa.page_scores_fp8(g, qs[l], summs[l], pt, sl, ws, scores=scores_buf)
+            else:
+                sa.page_scores(g, qs[l], summs[l], pt, sl, ws, scores=scores_buf)
             ev_sc[l][1].record()
 
     # capture: the step without events (headline), the step with per-phase events, and
@@ -378,15 +410,18 @@ def run_native(args, rank, world, dist):
     graph = torch.cuda.CUDAGraph()
     graph_ev = torch.cuda.CUDAGraph()
     graph_sc = torch.cuda.CUDAGraph()
+    # (fp8 summaries have no separate selection call: no per-phase pass)
     with torch.cuda.stream(stream):
-        step(True)                      # warm the stream before capture
+        if not F8:
+            step(True)                  # warm the stream before capture
         step_fused()
         score_only()
         torch.cuda.synchronize()
         with torch.cuda.graph(graph, stream=stream):
             step_fused()
-        with torch.cuda.graph(graph_ev, stream=stream):
-            step(True)
+        if not F8:
+            with torch.cuda.graph(graph_ev, stream=stream):
+                step(True)
         with torch.cuda.graph(graph_sc, stream=stream):
             score_only()
     torch.cuda.synchronize()
@@ -423,7 +458,7 @@ def run_native(args, rank, world, dist):
     n_ev = max(3, args.steps // 2)
     sc_ms = np.zeros(L_layers)
     with torch.cuda.stream(stream):
-        for _ in range(n_ev):
+        for _ in range(0 if F8 else n_ev):
             graph_ev.replay()
             torch.cuda.synchronize()
             for l in range(L_layers):
@@ -465,19 +500,21 @@ def run_native(args, rank, world, dist):
 
     if rank != 0:
         return 0
-    att_mean = float(att_ms.mean())
-    sel_mean = float(sel_ms.mean())
+    att_mean = None if F8 else float(att_ms.mean())
+    sel_mean = None if F8 else float(sel_ms.mean())
     sc_mean = float(sc_ms.mean())
     # page scoring: summaries + page-table entries + queries of one layer per launch
-    dom_kernel = "score_mla_kernel" if g.v_aliases_k else "score_stream_kernel"
+    dom_kernel = "score_mla_kernel" if g.v_aliases_k else (
+        "score_stream_kernel<fp8>" if F8 else "score_stream_kernel")
     dom_bytes, dom_ms = sel_b, sc_mean
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     cpu_v, cpu_done, cpu_t = (None, 0, 0.0)
     if world == 1:
-        cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds, R)
+        cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds, R, F8)
     # GQA: score, select (+ tail refresh), attention, merge; latent: tail refresh, query
     # sign split, tensor-core score, select, tensor-core attention, merge
-    launches_select = 4 if g.v_aliases_k else 2   # select half of one layer-call
+    # select half of one layer-call (fp8: the newest pages' records in a kernel of their own)
+    launches_select = 4 if g.v_aliases_k else (3 if F8 else 2)
     launches_attend = 2                           # attention + merge
     launches_per_step = n_sel_layers * launches_select + L_layers * launches_attend
     line = {
@@ -499,15 +536,17 @@ def run_native(args, rank, world, dist):
             "seq_len": int(case.seq_lens.max()), "page": P, "budget_tokens": case.budget,
             "sink": case.sink, "window": case.window, "layers_per_step": L_layers,
             "select_every": R,
-            "call": "sa_sparse_decode" if R == 1 else "sa_select_pages + sa_attend_selected",
+            "summaries": "fp8 e4m3 rounded outward" if F8 else "bf16",
+            "call": ("sa_sparse_decode_fp8" if F8 else "sa_sparse_decode") if R == 1 else
+                    "sa_select_pages + sa_attend_selected",
             "l2": "inputs larger than L2: %d distinct layer pools, %.2f GB touched per step"
                   % (L_layers, step_bytes / 1e9),
             "parallelism": "replicas (batch split), no collective" if world > 1 else "1 GPU",
             "step_hbm_gbs": step_gbs,
             "step_frac_of_hbm_peak": step_gbs / hbm_peak,
             "us_per_layer": ms_per_step * 1e3 / L_layers,
-            "select_pages_us_alone": sel_mean * 1e3,
-            "attend_selected_us_alone": att_mean * 1e3,
+            "select_pages_us_alone": None if sel_mean is None else sel_mean * 1e3,
+            "attend_selected_us_alone": None if att_mean is None else att_mean * 1e3,
             "page_scores_us_alone": sc_mean * 1e3,
             "summaries_us_alone": summ_ms * 1e3,
             "summaries_gbs_alone": summ_bytes / (summ_ms * 1e-3) / 1e9,

@@ -185,6 +185,44 @@ int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache, const
                      size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * fp8 summaries rounded outward (grouped-query geometry only; others return
+ * SA_ERR_UNSUPPORTED)  [SE hook-point paragraph: quantised KV (KIVI) listed next to
+ * Quest; the pages give no format].  Per (physical page, KV head) a record of
+ * 2*Dk + 16 bytes replaces the 4*Dk bytes of bf16 min/max:
+ *   summ8 [n_pool][Hkv][2*Dk + 16] uint8 = [Dk codes of min][Dk codes of max][int8 e]
+ *   [15 zero bytes].
+ * Codes are OCP FP8 E4M3 ("fn": bias 7, max finite 448, 0x7F/0xFF NaN never written):
+ * the min row rounded toward -inf and the max row toward +inf, of the bf16 min/max of
+ * sa_page_summaries scaled by 2^-e, where e is the smallest integer with
+ * max|value| * 2^-e <= 448 (e = 0 for an all-zero record).  Zero is the code 0x00.
+ * Decoded, code * 2^e <= kmin and >= kmax, so the page bound over the records is still
+ * an upper bound of every q.k on the page (never below the bf16 bound; equal to it
+ * when every scaled min/max is an exact code).  Bit-exact.
+ * sa_summary_fp8_record_bytes: 2*Dk + 16 for a supported geometry, else 0.
+ * sa_page_scores_fp8: the bound S of (2) over decoded records, fp32 (codes widened to
+ * bf16 exactly; products exact; fp32 accumulation), -inf beyond each sequence.
+ * sa_sparse_decode_fp8: sa_sparse_decode with the selection scored over fp8 records;
+ * attention still reads the bf16 K and V.  n_tail_refresh (0..16) re-encodes the
+ * newest pages' records from k_cache first (a kernel of its own).  Argument rules and
+ * workspace as for sa_sparse_decode (summ8 16-byte aligned).
+ * ------------------------------------------------------------------------------ */
+size_t sa_summary_fp8_record_bytes(const sa_geom* g);
+int sa_page_summaries_fp8(const sa_geom* g, const void* k_cache, const int32_t* page_table,
+                          const int32_t* seq_lens, void* summ8, void* stream);
+int sa_update_summaries_fp8(const sa_geom* g, const void* k_cache, const int32_t* page_table,
+                            const int32_t* seq_lens, int n_tail_pages, void* summ8,
+                            void* stream);
+int sa_page_scores_fp8(const sa_geom* g, const void* q, const void* summ8,
+                       const int32_t* page_table, const int32_t* seq_lens, float* scores,
+                       void* ws, size_t ws_bytes, void* stream);
+int sa_sparse_decode_fp8(const sa_geom* g, const void* q, const void* k_cache,
+                         const void* v_cache, void* summ8, const int32_t* page_table,
+                         const int32_t* seq_lens, int budget, int sink, int window,
+                         int n_tail_refresh, float scale, float* out, float* lse,
+                         int32_t* sel_out, int32_t* sel_count_out, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------------
  * Allocation-free sparse decode.  The pages have no counterpart to this call: it is an
  * engineering variant of sa_sparse_decode for callers that cannot hand the library a
  * workspace.  Arguments, results and argument errors are those of sa_sparse_decode

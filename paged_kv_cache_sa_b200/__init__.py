@@ -42,7 +42,9 @@ STATUS = {0: "SA_OK", -1: "SA_ERR_INVALID_ARG", -2: "SA_ERR_UNSUPPORTED", -3: "S
 EXPORTS = ["sa_status_string", "sa_version", "sa_decode_workspace_size", "sa_prune_workspace_size",
            "sa_workspace_init", "sa_workspace_status", "sa_page_summaries", "sa_update_summaries",
            "sa_page_scores", "sa_select_pages", "sa_sparse_decode", "sa_attend_selected",
-           "sa_prune_compact", "sa_sparse_decode_noalloc"]
+           "sa_prune_compact", "sa_sparse_decode_noalloc", "sa_summary_fp8_record_bytes",
+           "sa_page_summaries_fp8", "sa_update_summaries_fp8", "sa_page_scores_fp8",
+           "sa_sparse_decode_fp8"]
 
 
 class SaError(RuntimeError):
@@ -100,6 +102,12 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                               vp, vp, vp, vp, sz, vp], i32),
         "sa_sparse_decode_noalloc": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                       ctypes.c_float, vp, vp, vp, vp, vp, vp], i32),
+        "sa_summary_fp8_record_bytes": ([G], sz),
+        "sa_page_summaries_fp8": ([G, vp, vp, vp, vp, vp], i32),
+        "sa_update_summaries_fp8": ([G, vp, vp, vp, i32, vp, vp], i32),
+        "sa_page_scores_fp8": ([G, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "sa_sparse_decode_fp8": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
+                                  vp, vp, vp, vp, vp, sz, vp], i32),
         "sa_attend_selected": ([G, vp, vp, vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp,
                                 vp, sz, vp], i32),
         "sa_prune_compact": ([G, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, sz,
@@ -234,6 +242,66 @@ def sparse_decode(geom: Geometry, q, k_cache, v_cache, summ, page_table, seq_len
                                 int(window), int(n_tail_refresh), float(scale), _ptr(out),
                                 _ptr(lse), _ptr(sel_out), _ptr(sel_count_out), _ptr(ws.buf),
                                 ws.nbytes, _stream(stream)), "sa_sparse_decode")
+    return out, lse
+
+
+def summary_fp8_record_bytes(geom: Geometry) -> int:
+    g = geom.c()
+    return int(lib.sa_summary_fp8_record_bytes(ctypes.byref(g)))
+
+
+def empty_summaries_fp8(geom: Geometry, device=None) -> torch.Tensor:
+    """A zeroed fp8 record buffer [n_pool, Hkv, 2*Dk + 16] uint8."""
+    n = summary_fp8_record_bytes(geom)
+    if n == 0:
+        raise SaError(SA_ERR_UNSUPPORTED, "fp8 summaries")
+    return torch.zeros((geom.n_pool, geom.Hkv, n), dtype=torch.uint8, device=device or "cuda")
+
+
+def page_summaries_fp8(geom: Geometry, k_cache, page_table, seq_lens, summ8, stream=None):
+    g = geom.c()
+    _check(lib.sa_page_summaries_fp8(ctypes.byref(g), _ptr(k_cache), _ptr(page_table),
+                                     _ptr(seq_lens), _ptr(summ8), _stream(stream)),
+           "sa_page_summaries_fp8")
+    return summ8
+
+
+def update_summaries_fp8(geom: Geometry, k_cache, page_table, seq_lens, summ8,
+                         n_tail_pages: int = 1, stream=None):
+    g = geom.c()
+    _check(lib.sa_update_summaries_fp8(ctypes.byref(g), _ptr(k_cache), _ptr(page_table),
+                                       _ptr(seq_lens), int(n_tail_pages), _ptr(summ8),
+                                       _stream(stream)), "sa_update_summaries_fp8")
+    return summ8
+
+
+def page_scores_fp8(geom: Geometry, q, summ8, page_table, seq_lens, ws: Workspace, scores=None,
+                    stream=None):
+    if scores is None:
+        scores = torch.empty((geom.B, geom.Hkv, geom.max_pages), dtype=torch.float32,
+                             device=q.device)
+    g = geom.c()
+    _check(lib.sa_page_scores_fp8(ctypes.byref(g), _ptr(q), _ptr(summ8), _ptr(page_table),
+                                  _ptr(seq_lens), _ptr(scores), _ptr(ws.buf), ws.nbytes,
+                                  _stream(stream)), "sa_page_scores_fp8")
+    return scores
+
+
+def sparse_decode_fp8(geom: Geometry, q, k_cache, v_cache, summ8, page_table, seq_lens, budget,
+                      sink, window, scale, ws: Workspace, out=None, lse=None, sel_out=None,
+                      sel_count_out=None, n_tail_refresh: int = 0, stream=None):
+    dev = q.device
+    if out is None:
+        out = torch.empty((geom.B, geom.Hq, geom.Dv), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((geom.B, geom.Hq), dtype=torch.float32, device=dev)
+    g = geom.c()
+    _check(lib.sa_sparse_decode_fp8(ctypes.byref(g), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(summ8), _ptr(page_table), _ptr(seq_lens), int(budget),
+                                    int(sink), int(window), int(n_tail_refresh), float(scale),
+                                    _ptr(out), _ptr(lse), _ptr(sel_out), _ptr(sel_count_out),
+                                    _ptr(ws.buf), ws.nbytes, _stream(stream)),
+           "sa_sparse_decode_fp8")
     return out, lse
 
 

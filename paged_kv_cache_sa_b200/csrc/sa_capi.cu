@@ -354,6 +354,97 @@ SA_EXPORT int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_ca
   return run_attend(*g, plan, w, q, k_cache, vc, page_table, seq_lens, sel, cnt,
                     reinterpret_cast<int32_t*>(w + plan.off_phys), plan.K, scale, out, lse, s);
 }
+// ---- fp8 summaries rounded outward (grouped-query geometry) ---------------------------
+
+SA_EXPORT size_t sa_summary_fp8_record_bytes(const sa_geom* g) {
+  if (check_geom(g) != SA_OK || !is_gqa(*g) || !score_supported_fp8(*g)) return 0;
+  return 2 * (size_t)g->Dk + 16;
+}
+
+SA_EXPORT int sa_page_summaries_fp8(const sa_geom* g, const void* k_cache,
+                                    const int32_t* page_table, const int32_t* seq_lens,
+                                    void* summ8, void* stream) {
+  int st = check_geom(g);
+  if (st != SA_OK) return st;
+  if (!is_gqa(*g) || !score_supported_fp8(*g)) return SA_ERR_UNSUPPORTED;
+  if (!k_cache || !page_table || !seq_lens || !summ8) return SA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(summ8)) return SA_ERR_INVALID_ARG;
+  return cuda_status(launch_summaries_fp8(*g, k_cache, page_table, seq_lens, summ8, 0,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+SA_EXPORT int sa_update_summaries_fp8(const sa_geom* g, const void* k_cache,
+                                      const int32_t* page_table, const int32_t* seq_lens,
+                                      int n_tail_pages, void* summ8, void* stream) {
+  int st = check_geom(g);
+  if (st != SA_OK) return st;
+  if (!is_gqa(*g) || !score_supported_fp8(*g)) return SA_ERR_UNSUPPORTED;
+  if (!k_cache || !page_table || !seq_lens || !summ8 || n_tail_pages < 1)
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(summ8)) return SA_ERR_INVALID_ARG;
+  if (n_tail_pages > g->max_pages) n_tail_pages = g->max_pages;
+  return cuda_status(launch_summaries_fp8(*g, k_cache, page_table, seq_lens, summ8,
+                                          n_tail_pages, static_cast<cudaStream_t>(stream)));
+}
+
+SA_EXPORT int sa_page_scores_fp8(const sa_geom* g, const void* q, const void* summ8,
+                                 const int32_t* page_table, const int32_t* seq_lens,
+                                 float* scores, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_geom(g);
+  if (st != SA_OK) return st;
+  if (!is_gqa(*g) || !score_supported_fp8(*g)) return SA_ERR_UNSUPPORTED;
+  if (!q || !summ8 || !page_table || !seq_lens || !scores) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(summ8)) return SA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < 256 || !aligned16(ws)) return SA_ERR_WORKSPACE;
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  return cuda_status(launch_score(*g, q, summ8, page_table, seq_lens, scores,
+                                  score_ctas(*g, sm_count()), &hdr->status_bits,
+                                  static_cast<cudaStream_t>(stream), true));
+}
+
+SA_EXPORT int sa_sparse_decode_fp8(const sa_geom* g, const void* q, const void* k_cache,
+                                   const void* v_cache, void* summ8, const int32_t* page_table,
+                                   const int32_t* seq_lens, int budget, int sink, int window,
+                                   int n_tail_refresh, float scale, float* out, float* lse,
+                                   int32_t* sel_out, int32_t* sel_count_out, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  int st = check_geom(g);
+  if (st != SA_OK) return st;
+  if (!is_gqa(*g) || !score_supported_fp8(*g)) return SA_ERR_UNSUPPORTED;
+  if ((st = check_budget(*g, budget, sink, window)) != SA_OK) return st;
+  if (!q || !k_cache || !v_cache || !summ8 || !page_table || !seq_lens || !out || !lse)
+    return SA_ERR_INVALID_ARG;
+  if (n_tail_refresh < 0 || n_tail_refresh > 16) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(summ8))
+    return SA_ERR_INVALID_ARG;
+  if ((size_t)g->max_pages * 4 > 200 * 1024) return SA_ERR_UNSUPPORTED;
+  DecodePlan plan;
+  make_decode_plan(*g, budget, &plan);
+  if (!ws || ws_bytes < plan.total || !aligned16(ws)) return SA_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* status = &reinterpret_cast<WsHeader*>(w)->status_bits;
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + plan.off_sel);
+  int32_t* cnt = sel_count_out ? sel_count_out : reinterpret_cast<int32_t*>(w + plan.off_cnt);
+  int32_t* phys = reinterpret_cast<int32_t*>(w + plan.off_phys);
+  float* scores = reinterpret_cast<float*>(w + plan.off_scores);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // newest pages' records first (their own kernel), then the fp8 scoring, the selection
+  // (nothing left to refresh) and the attention over bf16 K and V
+  if (n_tail_refresh > 0 &&
+      (st = cuda_status(launch_summaries_fp8(*g, k_cache, page_table, seq_lens, summ8,
+                                             n_tail_refresh, s))) != SA_OK)
+    return st;
+  if ((st = cuda_status(launch_score(*g, q, summ8, page_table, seq_lens, scores,
+                                     plan.n_score_cta, status, s, true))) != SA_OK)
+    return st;
+  if ((st = cuda_status(launch_select(*g, q, nullptr, nullptr, 0, page_table, seq_lens, scores,
+                                      plan.K, sink / g->P, window / g->P, sel, cnt, phys, status,
+                                      s))) != SA_OK)
+    return st;
+  return run_attend(*g, plan, w, q, k_cache, v_cache, page_table, seq_lens, sel, cnt, phys,
+                    plan.K, scale, out, lse, s);
+}
+
 namespace sa {
 // Scratch of sa_sparse_decode_noalloc: a static device variable, one per device.
 static __device__ __align__(256) uint8_t g_static_scratch[SA_STATIC_SCRATCH_BYTES];

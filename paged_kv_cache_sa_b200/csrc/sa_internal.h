@@ -25,15 +25,21 @@ cudaError_t launch_summaries(const sa_geom& g, const void* k_cache, const int32_
                              const int32_t* seq_lens, void* summ, int n_tail,
                              cudaStream_t stream);
 
+// fp8 records [n_pool][Hkv][2 * Dk + 16] (grouped-query head dims 64 and 128)
+cudaError_t launch_summaries_fp8(const sa_geom& g, const void* k_cache,
+                                 const int32_t* page_table, const int32_t* seq_lens, void* summ8,
+                                 int n_tail, cudaStream_t stream);
+
 cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
                                 int n_tail, const int32_t* page_table, const int32_t* seq_lens,
                                 float* scores, int n_cta, int K, int sink_pages,
                                 int window_pages, int32_t* sel, int32_t* sel_count,
                                 int32_t* sel_phys, int32_t* status, cudaStream_t stream);
 
+// fp8: summ holds fp8 records (2 * Dk + 16 bytes per page and KV head)
 cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
                          const int32_t* page_table, const int32_t* seq_lens, float* scores,
-                         int n_cta, int32_t* status, cudaStream_t stream);
+                         int n_cta, int32_t* status, cudaStream_t stream, bool fp8 = false);
 cudaError_t launch_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
                           int n_tail, const int32_t* page_table, const int32_t* seq_lens,
                           float* scores, int K, int sink_pages, int window_pages, int32_t* sel,
@@ -56,6 +62,7 @@ cudaError_t launch_attend_mla(const sa_geom& g, const void* q, const void* kv,
 
 int score_ctas(const sa_geom& g, int sms);
 bool score_supported(const sa_geom& g);
+bool score_supported_fp8(const sa_geom& g);
 
 struct AttendCall {
   const void* q;

@@ -22,6 +22,11 @@
 // the same order, so the sum is unchanged) -- page slots are padded by 64 bytes so
 // those loads are free of bank conflicts -- and write the GQA-max score row.
 // HBM-bound: bytes per (page, KV head) = 2 * Dk * 2 (summary) + 4 / Hkv (page table).
+// fp8 records (score_stream_kernel<D, true>): the same tiles over [Dk codes of min |
+// Dk codes of max | int8 e | pad] records of 2 * Dk + 16 bytes, codes widened to bf16
+// exactly (every E4M3 value is a bf16 value) before the MMA, the record's 2^e applied
+// to the GQA-max score (a positive power of two commutes with the max).  Bytes per
+// (page, KV head): 2 * Dk + 16.
 //
 // Selection (select_kernel, one CTA per (sequence, KV head), launched programmatically
 // dependent on the scoring grid).  Before waiting for the scores it recomputes the
@@ -34,6 +39,10 @@
 // of the k-th best candidate and how many keys equal to T are needed; a final pass
 // marks forced pages, keys > T and the lowest-index keys == T, and two block scans
 // write the ascending list.  Deterministic.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
@@ -57,7 +66,21 @@ struct ScoreArgs {
   int B, Hq, Hkv, G, P, max_pages, n_pool;
   int HG, n_hg, WPS, NST;              // heads per tile, head groups, warp groups, stages
   int slot_bytes, q_off, stage_bytes;  // stage: [16][slot_bytes] page slots | q rows
+  int rec_bytes;                       // summary bytes per (page, KV head)
 };
+
+// Four E4M3 codes (bytes of w, lowest first) as two bf16x2 words, exactly: the
+// hardware e4m3x2 -> f16x2 conversion, then f16 -> f32 -> bf16 (no rounding anywhere:
+// every E4M3 value has at most 4 significant bits within the exponent range of both).
+__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const __half2 a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  const __half2 b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  const float2 fa = __half22float2(a), fb = __half22float2(b);
+  const __nv_bfloat162 ba = __floats2bfloat162_rn(fa.x, fa.y);
+  const __nv_bfloat162 bb = __floats2bfloat162_rn(fb.x, fb.y);
+  lo = *reinterpret_cast<const uint32_t*>(&ba);
+  hi = *reinterpret_cast<const uint32_t*>(&bb);
+}
 
 __device__ __forceinline__ void named_barrier_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -76,7 +99,7 @@ __device__ __forceinline__ int find_seq(const int* pre, int n, int u) {
   return lo;
 }
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const ScoreArgs a) {
   constexpr int J = D / 16;  // 16-byte chunks per lane of the 2*D-long contraction row
   extern __shared__ uint8_t smem_raw[];
@@ -188,7 +211,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
     named_barrier_sync(1, kScoreThreads);  // tables ready
 
     // ===================== producer warp: bulk-copy issue =====================
-    const uint32_t slot_data = (uint32_t)a.HG * 4 * D;  // one page's summaries of the group
+    const uint32_t slot_data = (uint32_t)a.HG * a.rec_bytes;  // one page's records of the group
     const uint32_t q_bytes = (uint32_t)a.HG * a.G * D * 2;
     uint64_t t_idle = 0;
     for (int k = 0; k < nt;) {
@@ -216,8 +239,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
       __syncwarp();
       if (lane < kTilePages && ((vm >> lane) & 1)) {
         const int ph = ptab[k * kTilePages + lane];
-        bulk_load(st + lane * a.slot_bytes, a.summ + ((size_t)ph * a.Hkv + hg * a.HG) * 4 * D,
-                  slot_data, &full_bar[s]);
+        bulk_load(st + lane * a.slot_bytes,
+                  a.summ + ((size_t)ph * a.Hkv + hg * a.HG) * (size_t)a.rec_bytes, slot_data,
+                  &full_bar[s]);
       } else if (lane == kTilePages) {
         bulk_load(st + a.q_off, a.q + ((size_t)b * a.Hq + (size_t)hg * a.HG * a.G) * D, q_bytes,
                   &full_bar[s]);
@@ -259,13 +283,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
         }
         // A: rows r and r + 8 of the tile (pages p0 + r, p0 + r + 8)
         const bool va = (vm >> r) & 1, vb = (vm >> (r + 8)) & 1;
-        const uint32_t rowa = st + r * a.slot_bytes + hh * 4 * D;
+        const uint32_t rowa = st + r * a.slot_bytes + hh * a.rec_bytes;
         const uint32_t rowb = rowa + 8 * a.slot_bytes;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-          const uint4 ra = va ? lds_v4(rowa + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
-          const uint4 rb = vb ? lds_v4(rowb + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
+          uint4 ra, rb;
+          if constexpr (F8) {
+            // chunk 4j + t of the contraction = 8 codes (channels of the same q chunk)
+            const uint2 ca = va ? lds_v2(rowa + (4 * j + t) * 8) : make_uint2(0, 0);
+            const uint2 cb = vb ? lds_v2(rowb + (4 * j + t) * 8) : make_uint2(0, 0);
+            e4m3x4_to_bf16(ca.x, ra.x, ra.y);
+            e4m3x4_to_bf16(ca.y, ra.z, ra.w);
+            e4m3x4_to_bf16(cb.x, rb.x, rb.y);
+            e4m3x4_to_bf16(cb.y, rb.z, rb.w);
+          } else {
+            ra = va ? lds_v4(rowa + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
+            rb = vb ? lds_v4(rowb + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
+          }
           mma_bf16_16816(acc, ra.x, rb.x, ra.y, rb.y, bq[j][0], bq[j][1]);
           mma_bf16_16816(acc, ra.z, rb.z, ra.w, rb.w, bq[j][2], bq[j][3]);
         }
@@ -276,6 +311,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
         m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
         m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
         m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+        if constexpr (F8) {
+          // the records' exponents (an invalid page scored 0 stays 0)
+          const uint8_t* sp = stages + (size_t)s * a.stage_bytes + hh * a.rec_bytes + 2 * D;
+          m0 = ldexpf(m0, (int)(int8_t)sp[r * a.slot_bytes]);
+          m1 = ldexpf(m1, (int)(int8_t)sp[(r + 8) * a.slot_bytes]);
+        }
         if (t == 0) {
           float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages + p0;
           if (r < np) srow[r] = m0;
@@ -686,23 +727,41 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-// Tile shape of the scoring grid for geometry g (see ScoreArgs).
-static void score_shape(const sa_geom& g, ScoreArgs* a) {
+// shared memory of the scoring grid besides its stages: alignment slack and tables
+static size_t score_table_bytes(const sa_geom& g) {
+  return 128 + (size_t)(2 * g.B + 1) * 4 + (size_t)kMaxTilesPerCta * kTilePages * 4 +
+         (size_t)5 * kMaxTilesPerCta * 4;
+}
+
+// Tile shape of the scoring grid for geometry g (see ScoreArgs); f8: fp8 records.
+static void score_shape(const sa_geom& g, ScoreArgs* a, bool f8 = false) {
   const int D = g.Dk;
-  int hg = 1;  // power of two dividing Hkv, at most 2 KB of summaries per page slot
+  int hg = 1;  // power of two dividing Hkv, at most 2 KB of bf16 summaries per page slot
   while (hg * 2 * 4 * D <= 2048 && g.Hkv % (hg * 2) == 0) hg *= 2;
   a->HG = hg;
   a->n_hg = g.Hkv / hg;
   a->WPS = kScoreConsumers / hg;
-  a->NST = a->WPS <= 4 ? 4 : 8;  // a multiple of WPS: one warp group per stage slot
-  a->slot_bytes = hg * 4 * D + kSlotPad;
+  if (!f8) {
+    a->rec_bytes = 4 * D;
+    a->NST = a->WPS <= 4 ? 4 : 8;  // a multiple of WPS: one warp group per stage slot
+    a->slot_bytes = hg * 4 * D + kSlotPad;
+  } else {
+    // half the bytes per stage: twice the stages in flight.  8-byte code loads of four
+    // page rows per half-warp are conflict-free when slots sit 32 B apart mod 128.
+    a->rec_bytes = 2 * D + 16;
+    a->NST = 8;
+    a->slot_bytes = ((hg * a->rec_bytes + 127) & ~127) + 32;
+  }
   a->q_off = kTilePages * a->slot_bytes;
   a->stage_bytes = (a->q_off + hg * (g.Hq / g.Hkv) * D * 2 + 127) & ~127;
+  // fp8: back to four stages when eight do not fit (large query groups)
+  if (f8 && a->WPS <= 4 &&
+      (size_t)8 * a->stage_bytes + score_table_bytes(g) > (size_t)kScoreSmemLimit)
+    a->NST = 4;
 }
 
 static size_t score_smem(const sa_geom& g, const ScoreArgs& a) {
-  return 128 + (size_t)a.NST * a.stage_bytes + (size_t)(2 * g.B + 1) * 4 +
-         (size_t)kMaxTilesPerCta * kTilePages * 4 + (size_t)5 * kMaxTilesPerCta * 4;
+  return (size_t)a.NST * a.stage_bytes + score_table_bytes(g);
 }
 
 int score_ctas(const sa_geom& g, int sms) {
@@ -722,9 +781,16 @@ bool score_supported(const sa_geom& g) {
   return score_smem(g, a) <= (size_t)kScoreSmemLimit;
 }
 
+bool score_supported_fp8(const sa_geom& g) {
+  if (!(g.Dk == 64 || g.Dk == 128)) return false;
+  ScoreArgs a;
+  score_shape(g, &a, true);
+  return score_smem(g, a) <= (size_t)kScoreSmemLimit;
+}
+
 static ScoreArgs make_score_args(const sa_geom& g, const void* q, const void* summ,
                                  const int32_t* page_table, const int32_t* seq_lens,
-                                 float* scores, int32_t* status) {
+                                 float* scores, int32_t* status, bool f8) {
   ScoreArgs a;
   a.q = static_cast<const uint16_t*>(q);
   a.summ = static_cast<const uint8_t*>(summ);
@@ -739,20 +805,22 @@ static ScoreArgs make_score_args(const sa_geom& g, const void* q, const void* su
   a.P = g.P;
   a.max_pages = g.max_pages;
   a.n_pool = g.n_pool;
-  score_shape(g, &a);
+  score_shape(g, &a, f8);
   return a;
 }
 
 cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
                          const int32_t* page_table, const int32_t* seq_lens, float* scores,
-                         int n_cta, int32_t* status, cudaStream_t stream) {
-  ScoreArgs a = make_score_args(g, q, summ, page_table, seq_lens, scores, status);
+                         int n_cta, int32_t* status, cudaStream_t stream, bool fp8) {
+  ScoreArgs a = make_score_args(g, q, summ, page_table, seq_lens, scores, status, fp8);
   const size_t smem = score_smem(g, a);
   const void* kern;
   if (g.Dk == 64)
-    kern = reinterpret_cast<const void*>(score_stream_kernel<64>);
+    kern = fp8 ? reinterpret_cast<const void*>(score_stream_kernel<64, true>)
+               : reinterpret_cast<const void*>(score_stream_kernel<64>);
   else if (g.Dk == 128)
-    kern = reinterpret_cast<const void*>(score_stream_kernel<128>);
+    kern = fp8 ? reinterpret_cast<const void*>(score_stream_kernel<128, true>)
+               : reinterpret_cast<const void*>(score_stream_kernel<128>);
   else
     return cudaErrorInvalidValue;
   cudaError_t e =

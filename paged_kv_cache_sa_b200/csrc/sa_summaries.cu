@@ -9,17 +9,75 @@
 // read it in 16-byte vectors, reduce with SIMD 16-bit min/max on an order key
 // (-0 < +0, bit-exact), then combine lanes with shuffles.  HBM-bound: bytes per
 // (page, head) = valid_tokens * Dk * 2 read + 2 * Dk * 2 written.
+//
+// fp8 records (grouped-query head dims).  The same min/max, then stored as OCP FP8
+// E4M3 codes rounded outward -- the min row toward -inf, the max row toward +inf --
+// after scaling the (page, head) record by 2^-e, e the smallest integer with
+// max|value| * 2^-e <= 448, the largest finite code.  Decoded values (code * 2^e) then
+// bracket every key of the page, so the page bound over them is still an upper bound
+// (the quantised-KV option the SparseEngine blog's hook-point paragraph lists next to
+// Quest; the pages give no format).  Record: [Dk codes min][Dk codes max][int8 e][15
+// zero bytes].  The encoder works on the bf16 bit fields, so no value is rounded before
+// the one outward step.
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
 namespace sa {
 
-// CPR = 16-byte chunks per key row (Dk / 8).
-template <int CPR>
+// Exponent of an fp8 record from the largest magnitude A (bf16 magnitude bits): with
+// A = f * 2^E, f in [0.5, 1), the smallest e with A * 2^-e <= 448 = 0.875 * 2^9 is E - 9
+// when f <= 0.875 and E - 8 otherwise; 0 for A = 0.
+__device__ __forceinline__ int fp8_record_exp(uint32_t amag) {
+  if (amag == 0) return 0;
+  int E;
+  const float f = frexpf(__uint_as_float(amag << 16), &E);
+  return f <= 0.875f ? E - 9 : E - 8;
+}
+
+// E4M3 code of (bf16 value v) * 2^-e rounded toward +inf (up) or -inf (!up), for
+// |v * 2^-e| <= 448.  v = S * 2^X exactly (S the 8-bit significand); the target binade
+// of floor(log2 |x|) = k has the step 2^(k-3), or 2^-9 below the normal range, and the
+// code of T steps of 2^q is 8 * (q + 9) + T (T = 16 carries into the next binade, and
+// subnormal T = 8 is the smallest normal).  Zero results are the code 0x00.
+__device__ __forceinline__ uint32_t e4m3_outward(uint32_t v, int e, bool up) {
+  const uint32_t mag = v & 0x7FFFu;
+  if (mag == 0) return 0u;
+  const bool neg = (v & 0x8000u) != 0;
+  const uint32_t E8 = mag >> 7, m7 = mag & 0x7Fu;
+  const uint32_t S = E8 ? (0x80u | m7) : m7;
+  const int X = (E8 ? (int)E8 : 1) - 134 - e;
+  const int k = 31 - __clz(S) + X;
+  const int q = max(k - 3, -9);
+  const int sh = X - q;
+  uint32_t T;
+  if (sh >= 0) {
+    T = S << sh;
+  } else {
+    const int r = -sh;
+    T = r >= 32 ? 0u : (S >> r);
+    const bool inexact = r >= 32 ? true : (S & ((1u << r) - 1u)) != 0u;
+    if (inexact && up != neg) ++T;  // the magnitude moves away from zero
+  }
+  const uint32_t code = 8u * (uint32_t)(q + 9) + T;
+  return code == 0u ? 0u : (neg ? (0x80u | code) : code);
+}
+
+// the four codes of the bf16 pairs (a, b) as bytes lo..hi of one word
+__device__ __forceinline__ uint32_t e4m3_pack(uint32_t a, uint32_t b, int e, bool up) {
+  return e4m3_outward(a & 0xFFFFu, e, up) | (e4m3_outward(a >> 16, e, up) << 8) |
+         (e4m3_outward(b & 0xFFFFu, e, up) << 16) | (e4m3_outward(b >> 16, e, up) << 24);
+}
+
+__device__ __forceinline__ uint32_t max_mag2(uint32_t m, uint32_t w) {
+  return max(m, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
+}
+
+// CPR = 16-byte chunks per key row (Dk / 8).  F8: write fp8 records (CPR 8 or 16).
+template <int CPR, bool F8 = false>
 __global__ void __launch_bounds__(256) summaries_kernel(const uint4* __restrict__ k_cache,
                                                         const int32_t* __restrict__ page_table,
                                                         const int32_t* __restrict__ seq_lens,
-                                                        uint4* __restrict__ summ, int Hkv, int P,
+                                                        void* __restrict__ summ_out, int Hkv, int P,
                                                         int max_pages, int n_pool, int n_tail) {
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
@@ -36,7 +94,7 @@ __global__ void __launch_bounds__(256) summaries_kernel(const uint4* __restrict_
   const int valid = min(P, L - lp * P);
   for (int h = threadIdx.x >> 5; h < Hkv; h += blockDim.x >> 5) {
   const uint4* blk = k_cache + ((size_t)phys * Hkv + h) * P * CPR;
-  uint4* out = summ + ((size_t)phys * Hkv + h) * 2 * CPR;
+  uint4* out = static_cast<uint4*>(summ_out) + ((size_t)phys * Hkv + h) * 2 * CPR;
 
   if constexpr (32 % CPR == 0) {
     // lanes split a row; each lane keeps one chunk index for the whole page
@@ -64,9 +122,26 @@ __global__ void __launch_bounds__(256) summaries_kernel(const uint4* __restrict_
       mx.z = __vmaxs2(mx.z, __shfl_xor_sync(0xffffffffu, mx.z, off));
       mx.w = __vmaxs2(mx.w, __shfl_xor_sync(0xffffffffu, mx.w, off));
     }
-    if (lane < CPR) {
-      out[c] = make_uint4(bf2_key(mn.x), bf2_key(mn.y), bf2_key(mn.z), bf2_key(mn.w));
-      out[CPR + c] = make_uint4(bf2_key(mx.x), bf2_key(mx.y), bf2_key(mx.z), bf2_key(mx.w));
+    const uint4 lo = make_uint4(bf2_key(mn.x), bf2_key(mn.y), bf2_key(mn.z), bf2_key(mn.w));
+    const uint4 hi = make_uint4(bf2_key(mx.x), bf2_key(mx.y), bf2_key(mx.z), bf2_key(mx.w));
+    if constexpr (F8) {
+      // every lane holds chunk lane % CPR: the warp max covers the whole record
+      uint32_t am = max_mag2(max_mag2(max_mag2(max_mag2(0u, lo.x), lo.y), lo.z), lo.w);
+      am = max_mag2(max_mag2(max_mag2(max_mag2(am, hi.x), hi.y), hi.z), hi.w);
+      am = __reduce_max_sync(0xffffffffu, am);
+      const int e = fp8_record_exp(am);
+      constexpr int D = CPR * 8;
+      uint8_t* rec = static_cast<uint8_t*>(summ_out) + ((size_t)phys * Hkv + h) * (2 * D + 16);
+      if (lane < CPR) {
+        *reinterpret_cast<uint2*>(rec + c * 8) =
+            make_uint2(e4m3_pack(lo.x, lo.y, e, false), e4m3_pack(lo.z, lo.w, e, false));
+        *reinterpret_cast<uint2*>(rec + D + c * 8) =
+            make_uint2(e4m3_pack(hi.x, hi.y, e, true), e4m3_pack(hi.z, hi.w, e, true));
+      }
+      if (lane == 0) *reinterpret_cast<uint4*>(rec + 2 * D) = make_uint4((uint32_t)e & 0xFFu, 0u, 0u, 0u);
+    } else if (lane < CPR) {
+      out[c] = lo;
+      out[CPR + c] = hi;
     }
   } else {
     // wide rows (latent keys): each lane owns chunks lane, lane+32, ... of every row
@@ -106,6 +181,29 @@ __global__ void __launch_bounds__(256) summaries_kernel(const uint4* __restrict_
   }  // heads
 }
 
+cudaError_t launch_summaries_fp8(const sa_geom& g, const void* k_cache,
+                                 const int32_t* page_table, const int32_t* seq_lens, void* summ8,
+                                 int n_tail, cudaStream_t stream) {
+  const int grid_x = n_tail > 0 ? n_tail : g.max_pages;
+  dim3 grid(grid_x, g.B);
+  dim3 block(32 * (g.Hkv < 8 ? g.Hkv : 8));
+  const uint4* k = static_cast<const uint4*>(k_cache);
+  switch (g.Dk) {
+    case 64:
+      summaries_kernel<8, true><<<grid, block, 0, stream>>>(k, page_table, seq_lens, summ8, g.Hkv,
+                                                            g.P, g.max_pages, g.n_pool, n_tail);
+      break;
+    case 128:
+      summaries_kernel<16, true><<<grid, block, 0, stream>>>(k, page_table, seq_lens, summ8,
+                                                             g.Hkv, g.P, g.max_pages, g.n_pool,
+                                                             n_tail);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_summaries(const sa_geom& g, const void* k_cache, const int32_t* page_table,
                              const int32_t* seq_lens, void* summ, int n_tail,
                              cudaStream_t stream) {
@@ -113,7 +211,7 @@ cudaError_t launch_summaries(const sa_geom& g, const void* k_cache, const int32_
   dim3 grid(grid_x, g.B);
   dim3 block(32 * (g.Hkv < 8 ? g.Hkv : 8));
   const uint4* k = static_cast<const uint4*>(k_cache);
-  uint4* s = static_cast<uint4*>(summ);
+  void* s = summ;
   switch (g.Dk) {
     case 64:
       summaries_kernel<8><<<grid, block, 0, stream>>>(k, page_table, seq_lens, s, g.Hkv, g.P,

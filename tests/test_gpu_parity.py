@@ -351,6 +351,119 @@ def test_attend_selected_reuses_indices():
     check_attention(out.cpu().numpy(), lse.cpu().numpy(), ro, rl)
 
 
+# ------------------------------------------------------------------------------------
+# fp8 summaries rounded outward: records bit-exact, scores and decode against the oracle
+# ------------------------------------------------------------------------------------
+
+FP8 = [
+    dict(wl="tiny", B=3, seq_lens=[4096, 700, 33], Hkv=2, Hq=8, poison="nan"),
+    dict(wl="tiny", B=2, seq_lens=[3000, 1], Hkv=4, Hq=32),
+    dict(wl="llama32k", B=2, L=(8192, 8192), seed=91),
+    dict(wl="ragged", B=2, L=(3000, 9000), seed=92, budget=1024, sink=128, window=256,
+         poison="nan"),
+]
+
+
+def _fp8_check(case, dc, s8, lse_rel=None):
+    g = dc.g
+    ref8 = oracle.page_summaries_fp8(case.geom, case.k_cache, case.page_table, case.seq_lens)
+    assert np.array_equal(s8.cpu().numpy(), ref8)
+    osc = oracle.page_scores_fp8(case.geom, case.q, ref8, case.page_table, case.seq_lens)
+    ws = sa.Workspace.for_decode(g, case.budget)
+    gsc = sa.page_scores_fp8(g, dc.q, s8, dc.pt, dc.sl, ws).cpu().numpy()
+    fin = np.isfinite(osc)
+    assert np.array_equal(fin, np.isfinite(gsc))
+    assert np.allclose(gsc[fin], osc[fin], rtol=1e-5, atol=1e-4)
+    K = case.budget // g.P
+    sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((g.B, g.Hkv), dtype=torch.int32, device="cuda")
+    out, lse = sa.sparse_decode_fp8(g, dc.q, dc.k, dc.v, s8, dc.pt, dc.sl, case.budget,
+                                    case.sink, case.window, case.scale, ws, sel_out=sel,
+                                    sel_count_out=cnt)
+    assert ws.status() == sa.SA_OK
+    gs, gc = sel.cpu().numpy(), cnt.cpu().numpy()
+    osel, ocnt = oracle.select_pages(case.geom, osc, case.seq_lens, case.budget, case.sink,
+                                     case.window)
+    tied = check_selection(case.geom, case.seq_lens, case.budget, case.sink, case.window, osc,
+                           osel, ocnt, gs, gc)
+    o, l = oracle.attend(case.geom, case.q, case.k_cache, case.v_cache, case.page_table,
+                         case.seq_lens, gs if tied else osel, ocnt, case.scale)
+    if lse_rel is None:
+        check_attention(out.cpu().numpy(), lse.cpu().numpy(), o, l)
+    else:
+        # logits far beyond 1e3: lse to fp32 relative accuracy, out as usual
+        gl = lse.cpu().numpy()
+        check_attention(out.cpu().numpy(), l, o, l)
+        assert np.array_equal(np.isfinite(gl), np.isfinite(l))
+        f = np.isfinite(l)
+        assert (np.abs(gl[f] - l[f]) <= lse_rel * np.abs(l[f]) + 1e-3).all()
+    return gsc
+
+
+@pytest.mark.parametrize("kw", FP8, ids=lambda kw: "%s-B%d" % (kw["wl"], kw["B"]))
+def test_fp8_summaries_scores_and_decode(kw):
+    kw = dict(kw)
+    case = synth.decode_case(kw.pop("wl"), **kw)
+    dc = DevCase(case)
+    g = dc.g
+    s8 = sa.empty_summaries_fp8(g)
+    sa.page_summaries_fp8(g, dc.k, dc.pt, dc.sl, s8)
+    gsc = _fp8_check(case, dc, s8)
+    # never below the bf16 bound of the same pages
+    sa.page_summaries(g, dc.k, dc.pt, dc.sl, dc.summ)
+    ws = sa.Workspace.for_decode(g, case.budget)
+    s16 = sa.page_scores(g, dc.q, dc.summ, dc.pt, dc.sl, ws).cpu().numpy()
+    fin = np.isfinite(s16)
+    assert (gsc[fin] >= s16[fin] - 1e-5 * np.abs(s16[fin]) - 1e-4).all()
+
+
+def test_fp8_records_extreme_magnitudes():
+    # pages scaled by powers of two from 2^-40 to 2^60: positive and negative record
+    # exponents, E4M3 subnormals, and codes at 448
+    case = synth.decode_case("tiny", B=2, seq_lens=[1600, 900], Hkv=2, Hq=8, seed=93)
+    k = synth.bf16_to_f32(case.k_cache).astype(np.float64)
+    pw = np.array([-40, -12, -3, 0, 5, 20, 60])
+    s = pw[np.arange(k.shape[0]) % len(pw)]
+    k = k * (2.0 ** s)[:, None, None, None]
+    k[0::5, :, :, 7] = 0.0           # all-zero channels
+    k[1::9] = 0.0                    # all-zero pages: e = 0
+    case = dataclasses.replace(case, k_cache=synth.f32_to_bf16(k.astype(np.float32)))
+    dc = DevCase(case)
+    s8 = sa.empty_summaries_fp8(dc.g)
+    sa.page_summaries_fp8(dc.g, dc.k, dc.pt, dc.sl, s8)
+    _fp8_check(case, dc, s8, lse_rel=1e-5)
+
+
+def test_fp8_tail_refresh_inside_decode():
+    case = synth.decode_case("llama32k", B=3, seq_lens=[4097, 3000, 2064], seed=94,
+                             poison="nan")
+    dc = DevCase(case)
+    g = dc.g
+    before = to_dev(np.maximum(case.seq_lens - 1, 0))
+    s8 = sa.empty_summaries_fp8(g)
+    sa.page_summaries_fp8(g, dc.k, dc.pt, before, s8)      # newest page stale
+    ws = sa.Workspace.for_decode(g, case.budget)
+    out, lse = sa.sparse_decode_fp8(g, dc.q, dc.k, dc.v, s8, dc.pt, dc.sl, case.budget,
+                                    case.sink, case.window, case.scale, ws, n_tail_refresh=1)
+    assert ws.status() == sa.SA_OK
+    ref = oracle.decode_fp8(case)
+    assert np.array_equal(s8.cpu().numpy(), ref["summ8"])
+    check_attention(out.cpu().numpy(), lse.cpu().numpy(), ref["out"], ref["lse"])
+    # update_summaries_fp8 alone gives the same records
+    s8b = sa.empty_summaries_fp8(g)
+    sa.page_summaries_fp8(g, dc.k, dc.pt, before, s8b)
+    sa.update_summaries_fp8(g, dc.k, dc.pt, dc.sl, s8b, n_tail_pages=1)
+    assert np.array_equal(s8b.cpu().numpy(), ref["summ8"])
+
+
+def test_fp8_rejects_the_latent_geometry():
+    case = synth.decode_case("mla", B=1, seq_lens=[640])
+    g = sa.Geometry.of(case.geom)
+    assert sa.summary_fp8_record_bytes(g) == 0
+    with pytest.raises(sa.SaError):
+        sa.empty_summaries_fp8(g)
+
+
 def test_cross_layer_reuse_of_physical_pages():
     # layer 0 selects and returns the physical pages of its selection; the next layer
     # (own q, K, V; the same page table and lengths) attends over those physical pages
