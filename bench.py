@@ -16,8 +16,10 @@ with no event inside it; a second graph with an event between the two halves of 
 layer gives the per-phase times behind "roofline" (events between kernels cost the
 programmatic overlap of neighbouring kernels, so that pass is slightly slower).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama32k|llama128k|ragged]
+  python bench.py [--gpus N] [--steps K] [--warmup W]
+                  [--workload llama32k|llama128k|ragged|mla|prune|tiny]
   python bench.py --select-every 4   (cross-layer reuse: select at every 4th layer only)
+  python bench.py --summaries fp8    (fp8 summaries rounded outward, sa_sparse_decode_fp8)
   python bench.py --impl reference ...   (the CPU oracle on a bounded sample)
 
 Under torchrun (N > 1) every rank runs its own batch on its own GPU (weak scaling,

@@ -1,0 +1,39 @@
+"""Host-side pieces of bench.py: the algorithmic byte count per layer-call (bf16 and fp8
+summaries) and the oracle's timed sample, on CPU."""
+
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def test_layer_bytes_by_summary_format():
+    case = synth.decode_case("llama32k", B=2, seq_lens=[4096, 1000], seed=3)
+    g = case.geom
+    cnt = np.full((g.B, g.Hkv), case.budget // g.P, dtype=np.int32)
+    cnt[1] = (1000 + g.P - 1) // g.P                      # short sequence: all its pages
+    s16, a16, u16 = bench.layer_bytes(g, case.seq_lens, cnt, g.P)
+    s8, a8, u8 = bench.layer_bytes(g, case.seq_lens, cnt, g.P, fp8=True)
+    nb = (4096 + 15) // 16 + (1000 + 15) // 16
+    other = nb * 4 + g.B * g.Hq * g.Dk * 2                 # page table + q
+    assert s16 - other == nb * g.Hkv * 4 * g.Dk            # bf16 min/max rows
+    assert s8 - other == nb * g.Hkv * (2 * g.Dk + 16)      # fp8 records
+    assert a16 == a8                                       # attention reads bf16 K, V alike
+    # K+V of the selected valid tokens: sequence 0 full pages, sequence 1 ends at 1000
+    tok = g.Hkv * (128 * 16 + 1000)
+    assert a16 == tok * 2 * g.Dk * 2 + g.B * g.Hq * g.Dk * 2 + g.B * g.Hq * (g.Dv * 4 + 4)
+    assert u16 - u8 == g.B * g.Hkv * (4 * g.Dk - (2 * g.Dk + 16))
+
+
+def test_oracle_sample_both_formats_and_reuse():
+    case = synth.decode_case("tiny", B=2, seq_lens=[4096, 700], Hkv=1, Hq=4)
+    for fp8 in (False, True):
+        for r in (1, 3):
+            v, done, t = bench.oracle_sample(case, 0.05, select_every=r, fp8=fp8)
+            assert done >= 1 and t > 0 and v > 0

@@ -33,7 +33,10 @@ def test_header_declares_the_expected_entry_points():
     for name in ("sa_page_summaries", "sa_update_summaries", "sa_select_pages",
                  "sa_sparse_decode", "sa_attend_selected", "sa_prune_compact",
                  "sa_decode_workspace_size", "sa_prune_workspace_size", "sa_workspace_init",
-                 "sa_workspace_status", "sa_status_string", "sa_version"):
+                 "sa_workspace_status", "sa_status_string", "sa_version", "sa_page_scores",
+                 "sa_sparse_decode_noalloc", "sa_summary_fp8_record_bytes",
+                 "sa_page_summaries_fp8", "sa_update_summaries_fp8", "sa_page_scores_fp8",
+                 "sa_sparse_decode_fp8"):
         assert name in decl
 
 
@@ -62,6 +65,31 @@ def test_binding_loads_and_sizes_workspaces(libpath):
     bad = sa.Geometry(B=8, Hq=32, Hkv=8, Dk=96, Dv=96, P=16, max_pages=2048, n_pool=16384)
     assert sa.decode_workspace_size(bad, 2048) == 0          # unsupported head dim
     assert sa.prune_workspace_size(g) > 256
+
+
+def test_fp8_record_size_and_host_checks(libpath):
+    import paged_kv_cache_sa_b200 as sa
+    g = sa.Geometry(B=8, Hq=32, Hkv=8, Dk=128, Dv=128, P=16, max_pages=2048, n_pool=16384)
+    assert sa.summary_fp8_record_bytes(g) == 2 * 128 + 16
+    g64 = sa.Geometry(B=2, Hq=32, Hkv=4, Dk=64, Dv=64, P=16, max_pages=64, n_pool=128)
+    assert sa.summary_fp8_record_bytes(g64) == 2 * 64 + 16
+    lat = sa.Geometry(B=2, Hq=128, Hkv=1, Dk=576, Dv=512, P=64, max_pages=64, n_pool=128,
+                      v_aliases_k=1)
+    assert sa.summary_fp8_record_bytes(lat) == 0
+    # argument errors come back before any CUDA call
+    c = lat.c()
+    dummy = ctypes.c_void_p(4096)
+    assert sa.lib.sa_page_summaries_fp8(ctypes.byref(c), dummy, dummy, dummy, dummy,
+                                        None) == sa.SA_ERR_UNSUPPORTED
+    c = g.c()
+    assert sa.lib.sa_page_summaries_fp8(ctypes.byref(c), None, dummy, dummy, dummy,
+                                        None) == sa.SA_ERR_INVALID_ARG
+    assert sa.lib.sa_sparse_decode_fp8(ctypes.byref(c), dummy, dummy, dummy, dummy, dummy, dummy,
+                                       2048, 64, 512, 0, 0.1, dummy, dummy, None, None, dummy,
+                                       16, None) == sa.SA_ERR_WORKSPACE
+    assert sa.lib.sa_sparse_decode_fp8(ctypes.byref(c), dummy, dummy, dummy, dummy, dummy, dummy,
+                                       2048, 64, 3000, 0, 0.1, dummy, dummy, None, None, dummy,
+                                       1 << 30, None) == sa.SA_ERR_INVALID_ARG
 
 
 def test_no_cpu_fallback_in_binding():
