@@ -34,11 +34,13 @@
 // appended tokens) and scores them; those scores replace the streamed ones, so the
 // scoring grid may read either version of those summaries.  Then it turns the scores
 // into order-preserving 32-bit keys in shared memory (forced pages get key 0, below
-// every real score) and runs an MSB-first 8-bit radix select (warp-aggregated
-// shared-memory histograms, one warp scans the 256 bins).  That gives the exact key T
-// of the k-th best candidate and how many keys equal to T are needed; a final pass
-// marks forced pages, keys > T and the lowest-index keys == T, and two block scans
-// write the ascending list.  Deterministic.
+// every real score) and runs an MSB-first radix select with 11-bit digits, starting at
+// the highest bit in which the candidates' keys differ (shared-memory histogram, block
+// scan over the bins).  It stops when the boundary bin is taken whole (threshold key),
+// or holds at most 256 candidates, which are then ranked exactly by (key desc, page
+// asc) and the winners marked; all-equal boundary keys take the lowest pages.  The
+// ascending list of forced and taken pages (and their physical ids) is written with
+// per-warp ballots and one block barrier.  Deterministic.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
