@@ -1,5 +1,7 @@
-// sa_mla.cu -- page scoring for the latent (MLA) geometry on the 5th-generation tensor
-// cores: 128 query heads share one 576-wide latent key per token.
+// sa_mla.cu -- the latent (MLA) geometry on the 5th-generation tensor cores: 128 query
+// heads share one 576-wide latent key per token (V = its first 512 channels).  This
+// file holds the page scoring (below) and the attention over the selected pages with
+// its chunk merge (second section); selection is the shared select_kernel.
 //
 // Method (the page bound of the SparseEngine blog's hook-point paragraph, Quest):
 //   S(b,p) = max over the 128 heads g of sum_c max(q_gc * kmax_c, q_gc * kmin_c)
