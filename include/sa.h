@@ -89,14 +89,13 @@ const char* sa_status_string(int status);
 int sa_version(void);
 
 /* ---------------------------------------------------------------------------------
- * Workspace.  One buffer per (stream, geometry, budget): calls on one stream with the
- * same geometry and budget may share it; calls that may run concurrently, or that use
- * another geometry or budget, need their own (or a fresh sa_workspace_init in between,
- * since the layout of its counters depends on the geometry).  It must be zeroed once
- * before first use (sa_workspace_init); afterwards the library keeps it consistent
- * (its arrival counters return to zero at the end of every call).  Its first 256 bytes
- * hold the status word.  A call that reported SA_ERR_TIMEOUT may leave counters
- * behind: zero the workspace again before reusing it.
+ * Workspace.  Zero it once before first use (sa_workspace_init).  Its first 256 bytes
+ * hold the status word, the only part that must start at zero; the rest is scratch that
+ * each call writes before it reads it (scores, the selection and its physical pages, the
+ * split-KV partial states), so no state carries from one call to the next.  One
+ * workspace therefore serves any geometry and budget whose sa_decode_workspace_size it
+ * covers.  Calls that use one workspace must not overlap in time (use one per stream, or
+ * order the streams).
  * ------------------------------------------------------------------------------ */
 
 /* Bytes needed by sa_select_pages / sa_sparse_decode / sa_attend_selected for this
@@ -176,7 +175,9 @@ int sa_select_pages(const sa_geom* g, const void* q, void* summ, const int32_t* 
  *   hq / G;  out[b][hq] = sum_t softmax(x)_t v_t;  lse[b][hq] = log sum_t exp(x_t).
  * A sequence with seq_len 0 gives out = 0, lse = -inf.  bf16 inputs, fp32
  * accumulation.  sel_out / sel_count_out (nullable) receive the selection;
- * n_tail_refresh as in sa_select_pages.
+ * n_tail_refresh as in sa_select_pages (a refreshed page must not be shared with another
+ * sequence of the same call: that sequence's scoring may read either version of its
+ * summary).
  * ------------------------------------------------------------------------------ */
 int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache, const void* v_cache,
                      void* summ, const int32_t* page_table, const int32_t* seq_lens, int budget,
@@ -232,13 +233,20 @@ int sa_sparse_decode_fp8(const sa_geom* g, const void* q, const void* k_cache,
  *  - Limit: a geometry and budget whose sa_decode_workspace_size exceeds
  *    SA_STATIC_SCRATCH_BYTES is rejected with SA_ERR_WORKSPACE before any launch
  *    (Llama-3.1-8B geometry, batch 8, 128K tokens, budget 2048 needs about 8 MB).
+ *    The latent geometry at 16 sequences of 64K tokens with budget 2048 needs about
+ *    38 MB and is therefore refused; 8 such sequences fit.
  *  - Setup: the first call on a device, with that device current, looks the scratch up
- *    with cudaGetSymbolAddress and zeroes its status word synchronously; make that
- *    first call before any stream capture.
- *  - Zeroing: only the scratch's status word must start at zero; every call clears it
- *    again on `stream` after its kernels.
+ *    with cudaGetSymbolAddress (a host-side lookup, no device work); make that first
+ *    call before any stream capture.  The address is cached per device for the life of
+ *    the process: resetting a device (cudaDeviceReset) is not supported afterwards.
+ *  - Zeroing: the module's load zero-fills the scratch.  Every call clears the status
+ *    word on `stream` before its first launch; the rest of the header (the single-launch
+ *    decode's cursor, CTA count and call tag) must carry over from call to call and is
+ *    kept consistent by the kernels themselves.
  *  - status_out (nullable, device int32): receives, on `stream`, the bit-OR of the
- *    device-detected errors of this call ((1 << -status) per error, 0 when none).
+ *    device-detected errors of this call ((1 << -status) per error, 0 when none).  With
+ *    status_out NULL those errors are dropped: the next call clears the word, and no
+ *    other call reads the scratch's status.
  *  - Concurrency: the scratch is shared by all calls on a device.  Calls that can
  *    overlap in time (other streams, other host threads) race on it; the caller must
  *    serialise them.

@@ -60,8 +60,9 @@ bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan) {
   DecodePlan p{};
   p.K = budget / g.P;
   p.G = g.Hq / g.Hkv;
-  p.n_cta = attend_ctas(g, p.K, sm_count());
-  p.n_score_cta = score_ctas(g, sm_count());
+  p.n_sm = sm_count();
+  p.n_cta = attend_ctas(g, p.K, p.n_sm);
+  p.n_score_cta = score_ctas(g, p.n_sm);
   size_t off = 256;  // status header
   p.off_scores = off;
   off += up256((size_t)g.B * g.Hkv * g.max_pages * 4);
@@ -109,6 +110,23 @@ bool encode_rows_tmap(void* tmap_out, const void* base, uint64_t inner_elems, ui
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(static_cast<CUtensorMap*>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D view of a [rows][128] bf16 pool as (64 channels, rows, 2 halves of a row): one box
+// of {64, box_rows, 2} lands as [half][row][64] with the 128-byte swizzle, the layout of
+// two 2-D boxes of {64, box_rows}.
+bool encode_rows3_tmap(void* tmap_out, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, 2};
+  cuuint64_t strides[2] = {256, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(static_cast<CUtensorMap*>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                   const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -452,8 +470,8 @@ constexpr int kMaxDevices = 64;
 static void* g_scratch_addr[kMaxDevices];
 static std::mutex g_scratch_mu;
 
-// Device address of the current device's scratch; looked up (and its status word
-// zeroed) on the first call for that device.
+// Device address of the current device's scratch, looked up on the first call for that
+// device.  The module's load zero-fills the array, so no clearing is needed here.
 static int static_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
@@ -462,7 +480,6 @@ static int static_scratch(void** out) {
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return SA_ERR_CUDA;
-    if (cudaMemset(p, 0, sizeof(WsHeader)) != cudaSuccess) return SA_ERR_CUDA;
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -484,6 +501,9 @@ SA_EXPORT int sa_sparse_decode_noalloc(const sa_geom* g, const void* q, const vo
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != SA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // a fresh status word (and abort flag) for this call, before its first launch, so that a
+  // call that failed half-way leaves nothing behind for the next one
+  if (cudaMemsetAsync(scratch, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return SA_ERR_CUDA;
   st = sa_sparse_decode(g, q, k_cache, v_cache, summ, page_table, seq_lens, budget, sink, window,
                         n_tail_refresh, scale, out, lse, sel_out, sel_count_out, scratch,
                         SA_STATIC_SCRATCH_BYTES, stream);
@@ -492,7 +512,7 @@ SA_EXPORT int sa_sparse_decode_noalloc(const sa_geom* g, const void* q, const vo
       cudaMemcpyAsync(status_out, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
           cudaSuccess)
     return SA_ERR_CUDA;
-  return cuda_status(cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s));
+  return SA_OK;
 }
 
 SA_EXPORT int sa_prune_compact(const sa_geom* g, const void* k_cache, const void* v_cache,

@@ -15,6 +15,7 @@ struct DecodePlan {
   int G;      // query heads per KV head
   int n_cta;        // attention CTAs (one per SM, more for very large selections)
   int n_score_cta;  // scoring CTAs (one per SM, more for very long sequences)
+  int n_sm;         // streaming multiprocessors of the device
   size_t off_scores, off_sel, off_cnt, off_phys, off_pre, off_part, off_qs, total;
 };
 
@@ -101,5 +102,7 @@ size_t prune_workspace_bytes(const sa_geom& g);
 // TMA descriptor encoder from the driver (resolved once through the runtime).
 bool encode_rows_tmap(void* tmap_out, const void* base, uint64_t inner_elems, uint64_t rows,
                       uint32_t box_inner, uint32_t box_rows);
+// 3-D descriptor of a [rows][128] bf16 pool: one box = box_rows rows, both 128-byte halves.
+bool encode_rows3_tmap(void* tmap_out, const void* base, uint64_t rows, uint32_t box_rows);
 
 }  // namespace sa

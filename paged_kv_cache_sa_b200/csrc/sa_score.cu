@@ -47,6 +47,7 @@
 
 #include "sa_common.cuh"
 #include "sa_internal.h"
+#include "sa_select.cuh"
 
 namespace sa {
 
@@ -347,113 +348,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
   }
 }
 
-template <int NT>
-__device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += u;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int wv = lane < NT / 32 ? warp_tot[lane] : 0;
-    int wi = wv;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, wi, off);
-      if (lane >= off) wi += u;
-    }
-    if (lane < NT / 32) warp_tot[lane] = wi - wv;  // exclusive warp offsets
-    if (lane == 31) warp_tot[NT / 32] = wi;        // block total
-  }
-  __syncthreads();
-  const int res = warp_tot[warp] + incl - v;
-  *total = warp_tot[NT / 32];
-  __syncthreads();
-  return res;
-}
-
-// Recompute the summary of one (physical page, KV head) from K (one warp), store it,
-// and return in every lane its score for the G query heads at qh (max over heads).
-template <int D>
-__device__ float warp_refresh_and_score(const uint4* __restrict__ k_cache,
-                                        uint4* __restrict__ summ, const uint16_t* qh, int G,
-                                        int phys, int h, int Hkv, int P, int valid, int lane) {
-  constexpr int CPR = D / 8;     // 8 or 16 chunks per row
-  constexpr int RPI = 32 / CPR;  // rows per warp iteration
-  const int c = lane % CPR;
-  const uint4* blk = k_cache + ((size_t)phys * Hkv + h) * P * CPR;
-  uint4 mn = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
-  uint4 mx = make_uint4(0x80008000u, 0x80008000u, 0x80008000u, 0x80008000u);
-  // query rows first: independent of K, so their loads are in flight with K's
-  uint4 qv[8];
-#pragma unroll
-  for (int g = 0; g < 8; ++g)
-    qv[g] = (g < G && lane < CPR) ? *reinterpret_cast<const uint4*>(qh + (size_t)g * D + c * 8)
-                                  : make_uint4(0, 0, 0, 0);
-#pragma unroll 4
-  for (int t = lane / CPR; t < valid; t += RPI) {
-    const uint4 v = __ldcg(blk + (size_t)t * CPR + c);
-    const uint32_t k0 = bf2_key(v.x), k1 = bf2_key(v.y), k2 = bf2_key(v.z), k3 = bf2_key(v.w);
-    mn.x = __vmins2(mn.x, k0); mn.y = __vmins2(mn.y, k1);
-    mn.z = __vmins2(mn.z, k2); mn.w = __vmins2(mn.w, k3);
-    mx.x = __vmaxs2(mx.x, k0); mx.y = __vmaxs2(mx.y, k1);
-    mx.z = __vmaxs2(mx.z, k2); mx.w = __vmaxs2(mx.w, k3);
-  }
-#pragma unroll
-  for (int off = CPR; off < 32; off <<= 1) {
-    mn.x = __vmins2(mn.x, __shfl_xor_sync(0xffffffffu, mn.x, off));
-    mn.y = __vmins2(mn.y, __shfl_xor_sync(0xffffffffu, mn.y, off));
-    mn.z = __vmins2(mn.z, __shfl_xor_sync(0xffffffffu, mn.z, off));
-    mn.w = __vmins2(mn.w, __shfl_xor_sync(0xffffffffu, mn.w, off));
-    mx.x = __vmaxs2(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, off));
-    mx.y = __vmaxs2(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, off));
-    mx.z = __vmaxs2(mx.z, __shfl_xor_sync(0xffffffffu, mx.z, off));
-    mx.w = __vmaxs2(mx.w, __shfl_xor_sync(0xffffffffu, mx.w, off));
-  }
-  const uint4 kmin = make_uint4(bf2_key(mn.x), bf2_key(mn.y), bf2_key(mn.z), bf2_key(mn.w));
-  const uint4 kmax = make_uint4(bf2_key(mx.x), bf2_key(mx.y), bf2_key(mx.z), bf2_key(mx.w));
-  uint4* out = summ + ((size_t)phys * Hkv + h) * 2 * CPR;
-  if (lane < CPR) {
-    __stcg(out + c, kmin);
-    __stcg(out + CPR + c, kmax);
-  }
-  const uint32_t lo[4] = {kmin.x, kmin.y, kmin.z, kmin.w};
-  const uint32_t hi[4] = {kmax.x, kmax.y, kmax.z, kmax.w};
-  float best = -INFINITY;
-#pragma unroll
-  for (int g = 0; g < 8; ++g) {
-    if (g >= G) break;
-    const uint32_t qw[4] = {qv[g].x, qv[g].y, qv[g].z, qv[g].w};
-    float part = 0.f;
-    if (lane < CPR) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const float qf = __uint_as_float(hf ? (qw[e] & 0xFFFF0000u) : (qw[e] << 16));
-          const float a0 = __uint_as_float(hf ? (lo[e] & 0xFFFF0000u) : (lo[e] << 16));
-          const float a1 = __uint_as_float(hf ? (hi[e] & 0xFFFF0000u) : (hi[e] << 16));
-          part += fmaxf(qf * a1, qf * a0);
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    best = fmaxf(best, part);
-  }
-  return best;
-}
-
-constexpr int kMaxTail = 16;
-constexpr int kHistBits = 11;  // digit of the one-pass histogram
-constexpr int kHistBins = 1 << kHistBits;
-constexpr int kBinCap = 256;             // boundary-bin size ranked exactly
-constexpr uint32_t kWin = 0xFFFFFFFFu;   // marks a candidate taken from the boundary bin
-
 struct SelectArgs {
   const uint16_t* q;
   uint4* summ;
@@ -472,13 +366,15 @@ struct SelectArgs {
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs a) {
   constexpr int NT = kSelectThreads;
+  using Bar = SelBar<-1, NT>;
   extern __shared__ uint32_t keys[];  // [max_pages] keys, then [max_pages] page table
   __shared__ uint32_t hist[kHistBins];
-  __shared__ uint32_t sh_bin, sh_above, red[2 * (NT / 32)];
+  __shared__ uint32_t misc[4], red[2 * (NT / 32)];
   __shared__ uint32_t bin_key[kBinCap];
   __shared__ int bin_page[kBinCap];
-  __shared__ int warp_tot[NT / 32 + 1], sh_n;
+  __shared__ int warp_tot[NT / 32 + 1];
   __shared__ float tail_score[kMaxTail];
+  const SelScratch sh{hist, bin_key, bin_page, warp_tot, red, misc};
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x, b = blockIdx.y;
   const int G = a.Hq / a.Hkv;
@@ -549,128 +445,11 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
       }
     }
   }
-  kmn = __reduce_min_sync(0xffffffffu, kmn);
-  kmx = __reduce_max_sync(0xffffffffu, kmx);
-  if (lane == 0) {
-    red[warp] = kmn;
-    red[NT / 32 + warp] = kmx;
-  }
-  __syncthreads();
-  kmn = 0xFFFFFFFFu;
-  kmx = 0u;
-#pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    kmn = min(kmn, red[w]);
-    kmx = max(kmx, red[NT / 32 + w]);
-  }
+  block_key_range<NT, Bar>(kmn, kmx, red);
 
-  // 4. threshold: a candidate is taken when its key >= thr or it was marked kWin.
-  // MSB-first radix select with 11-bit digits starting at the highest bit in which the
-  // candidates differ (the bits above are common to all of them); it stops as soon as
-  // the boundary bin is wholly taken or small enough to rank exactly.
-  const int k_rem0 = K - a.s_pages - a.w_pages;  // < number of candidates here
-  uint64_t thr = 1ull << 32;                      // above every key: forced pages only
-  if (k_rem0 > 0) {
-    const uint32_t diff = kmn ^ kmx;
-    int hi = diff ? 31 - __clz(diff) : -1;  // highest undecided bit
-    uint32_t pmask;                         // bits decided so far (above hi)
-    if (hi < 0)
-      pmask = 0xFFFFFFFFu;  // all candidates are equal
-    else if (hi == 31)
-      pmask = 0u;
-    else
-      pmask = ~((2u << hi) - 1u);
-    uint32_t pval = kmn & pmask;
-    int k_need = k_rem0;
-    int state = 0;  // 0: go on, 1: thr set, 2: tie on the full key
-    while (state == 0) {
-      if (hi < 0) {
-        state = 2;
-        break;
-      }
-      const int lo = max(0, hi - (kHistBits - 1));
-      const uint32_t dmask = (2u << (hi - lo)) - 1u;
-      for (int i = tid; i < kHistBins; i += NT) hist[i] = 0;
-      __syncthreads();
-      for (int p = tid; p < nb; p += NT) {
-        const uint32_t key = keys[p];
-        if (!(p < a.s_pages || p >= wbeg) && (key & pmask) == pval)
-          atomicAdd(&hist[(key >> lo) & dmask], 1u);
-      }
-      __syncthreads();
-      // bins owned 8 per thread; candidates in bins above each thread's range
-      constexpr int BPT = kHistBins / NT;
-      int mine = 0;
-#pragma unroll
-      for (int i = 0; i < BPT; ++i) mine += hist[tid * BPT + i];
-      int total;
-      const int below = block_excl_scan<NT>(mine, warp_tot, &total);
-      int run = total - below - mine;
-      for (int i = BPT - 1; i >= 0; --i) {
-        const int cnt = hist[tid * BPT + i];
-        if (run < k_need && run + cnt >= k_need) {
-          sh_bin = tid * BPT + i;
-          sh_above = run;
-        }
-        run += cnt;
-      }
-      __syncthreads();
-      const uint32_t bstar = sh_bin;
-      k_need -= (int)sh_above;
-      const int nbin = hist[bstar];
-      pval |= bstar << lo;
-      pmask |= dmask << lo;
-      if (nbin == k_need) {  // the whole boundary bin is taken
-        thr = pval;
-        state = 1;
-      } else if (nbin <= kBinCap) {
-        // exact ranking inside the boundary bin: larger key first, then lower page
-        if (tid == 0) sh_n = 0;
-        __syncthreads();
-        for (int p = tid; p < nb; p += NT) {
-          const uint32_t key = keys[p];
-          if (!(p < a.s_pages || p >= wbeg) && (key & pmask) == pval) {
-            const int i = atomicAdd(&sh_n, 1);
-            bin_key[i] = key;
-            bin_page[i] = p;
-          }
-        }
-        __syncthreads();
-        if (tid < nbin) {
-          const uint32_t key = bin_key[tid];
-          const int pg = bin_page[tid];
-          int rank = 0;
-          for (int j = 0; j < nbin; ++j) {
-            const uint32_t kj = bin_key[j];
-            rank += kj > key || (kj == key && bin_page[j] < pg);
-          }
-          if (rank < k_need) keys[pg] = kWin;
-        }
-        thr = (uint64_t)pval + (1ull << lo);
-        state = 1;
-      }
-      hi = lo - 1;
-      __syncthreads();
-    }
-    if (state == 2) {
-      // the boundary keys are all equal to T = pval: take the lowest-index ones
-      const uint32_t T = pval;
-      const int seg = (nb + NT - 1) / NT;
-      const int beg = min(nb, tid * seg), end = min(nb, beg + seg);
-      int n_eq = 0;
-      for (int p = beg; p < end; ++p) n_eq += !(p < a.s_pages || p >= wbeg) && keys[p] == T;
-      int tot;
-      int er = block_excl_scan<NT>(n_eq, warp_tot, &tot);
-      for (int p = beg; p < end; ++p) {
-        if (!(p < a.s_pages || p >= wbeg) && keys[p] == T) {
-          if (er < k_need) keys[p] = kWin;
-          ++er;
-        }
-      }
-      thr = (uint64_t)T + 1;
-      __syncthreads();
-    }
-  }
+  // 4. threshold: a candidate is taken when its key >= thr or it was marked kWin
+  const uint64_t thr = radix_select_threshold<NT, Bar>(keys, nb, a.s_pages, wbeg,
+                                                       K - a.s_pages - a.w_pages, kmn, kmx, sh);
 
   // 5. ascending list: forced pages and taken candidates.  Each warp owns a contiguous
   // run of pages (a multiple of 32) and compacts it with ballots; one block barrier
