@@ -54,7 +54,7 @@ namespace sa {
 constexpr int kTilePages = 16;  // pages per tile: the M side of one MMA
 constexpr int kScoreConsumers = 8;
 constexpr int kScoreThreads = (kScoreConsumers + 1) * 32;
-constexpr int kMaxTilesPerCta = 128;
+constexpr int kMaxTilesPerCta = 64;
 constexpr int kSlotPad = 64;  // odd multiple of 64 B between page slots: no bank conflicts
 constexpr int kSelectThreads = 256;
 constexpr int kScoreSmemLimit = 227 * 1024;
@@ -515,17 +515,39 @@ static size_t score_table_bytes(const sa_geom& g) {
 }
 
 // Tile shape of the scoring grid for geometry g (see ScoreArgs); f8: fp8 records.
+// bf16: up to 8 KV heads per page slot (one 4 KB bulk copy per page at Dk = 128), as many
+// stages as fit (a page slot is padded by 64 B when that still leaves the same number of
+// stages: conflict-free fragment loads).
 static void score_shape(const sa_geom& g, ScoreArgs* a, bool f8 = false) {
   const int D = g.Dk;
-  int hg = 1;  // power of two dividing Hkv, at most 2 KB of bf16 summaries per page slot
-  while (hg * 2 * 4 * D <= 2048 && g.Hkv % (hg * 2) == 0) hg *= 2;
+  const int G = g.Hq / g.Hkv;
+  int hg = 1;
+  if (!f8) {
+    while (hg < kScoreConsumers && g.Hkv % (hg * 2) == 0) hg *= 2;
+  } else {
+    // power of two dividing Hkv, at most 2 KB of bf16-equivalent summaries per slot
+    while (hg * 2 * 4 * D <= 2048 && g.Hkv % (hg * 2) == 0) hg *= 2;
+  }
   a->HG = hg;
   a->n_hg = g.Hkv / hg;
   a->WPS = kScoreConsumers / hg;
+  const size_t limit = (size_t)kScoreSmemLimit - score_table_bytes(g);
   if (!f8) {
     a->rec_bytes = 4 * D;
-    a->NST = a->WPS <= 4 ? 4 : 8;  // a multiple of WPS: one warp group per stage slot
-    a->slot_bytes = hg * 4 * D + kSlotPad;
+    const int q_bytes = hg * G * D * 2;
+    int best = 0;
+    for (int pad = kSlotPad; pad >= 0; pad -= kSlotPad) {
+      const int slot = hg * 4 * D + pad;
+      const int stage = (kTilePages * slot + q_bytes + 127) & ~127;
+      int nst = (int)(limit / stage);
+      if (nst > 8) nst = 8;
+      nst -= nst % a->WPS;  // a multiple of WPS: one warp group per stage slot
+      if (nst > best) {
+        best = nst;
+        a->slot_bytes = slot;
+      }
+    }
+    a->NST = best;
   } else {
     // half the bytes per stage: twice the stages in flight.  8-byte code loads of four
     // page rows per half-warp are conflict-free when slots sit 32 B apart mod 128.
@@ -534,7 +556,7 @@ static void score_shape(const sa_geom& g, ScoreArgs* a, bool f8 = false) {
     a->slot_bytes = ((hg * a->rec_bytes + 127) & ~127) + 32;
   }
   a->q_off = kTilePages * a->slot_bytes;
-  a->stage_bytes = (a->q_off + hg * (g.Hq / g.Hkv) * D * 2 + 127) & ~127;
+  a->stage_bytes = (a->q_off + hg * G * D * 2 + 127) & ~127;
   // fp8: back to four stages when eight do not fit (large query groups)
   if (f8 && a->WPS <= 4 &&
       (size_t)8 * a->stage_bytes + score_table_bytes(g) > (size_t)kScoreSmemLimit)
@@ -559,7 +581,7 @@ bool score_supported(const sa_geom& g) {
   if (!(g.Dk == 64 || g.Dk == 128)) return false;
   ScoreArgs a;
   score_shape(g, &a);
-  return score_smem(g, a) <= (size_t)kScoreSmemLimit;
+  return a.NST >= 2 && score_smem(g, a) <= (size_t)kScoreSmemLimit;
 }
 
 bool score_supported_fp8(const sa_geom& g) {
