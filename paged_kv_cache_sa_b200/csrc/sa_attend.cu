@@ -252,6 +252,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     const int j_end = lane < NC ? min(nu, j + W) : 0;
     int k = 0;  // units issued to consumer warp `lane`
     uint64_t t_idle = 0;
+    const uint64_t ef = l2_evict_first();
     for (;;) {
       const bool busy = j < j_end;
       bool issued = false;
@@ -265,8 +266,10 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
             mbar_arrive_expect_tx(&full_bar[st], S::STAGE_BYTES);
 #pragma unroll
             for (int hf = 0; hf < S::HALVES; ++hf) {
-              tma_load_2d(kdst + hf * S::HALF_BYTES, &kmap, hf * 64, row, &full_bar[st]);
-              tma_load_2d(vdst + hf * S::HALF_BYTES, &vmap, hf * 64, row, &full_bar[st]);
+              tma_load_2d_hint(kdst + hf * S::HALF_BYTES, &kmap, hf * 64, row, &full_bar[st],
+                               ef);
+              tma_load_2d_hint(vdst + hf * S::HALF_BYTES, &vmap, hf * 64, row, &full_bar[st],
+                               ef);
             }
           } else {
             mbar_arrive(&full_bar[st]);

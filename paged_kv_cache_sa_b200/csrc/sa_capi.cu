@@ -224,9 +224,8 @@ static int run_select(const sa_geom& g, const DecodePlan& plan, uint8_t* w, cons
     int st = cuda_status(launch_score_mla(g, q, summ, w + plan.off_qs, page_table, seq_lens,
                                           scores, &hdr->status_bits, s));
     if (st != SA_OK) return st;
-    return cuda_status(launch_select(g, q, summ, nullptr, 0, page_table, seq_lens, scores, plan.K,
-                                     sink / g.P, window / g.P, sel, cnt, phys, &hdr->status_bits,
-                                     s));
+    return cuda_status(launch_select(g, page_table, seq_lens, scores, plan.K, sink / g.P,
+                                     window / g.P, sel, cnt, phys, &hdr->status_bits, s));
   }
   if (!is_gqa(g)) return SA_ERR_UNSUPPORTED;
   return cuda_status(launch_score_select(
@@ -455,9 +454,8 @@ SA_EXPORT int sa_sparse_decode_fp8(const sa_geom* g, const void* q, const void* 
   if ((st = cuda_status(launch_score(*g, q, summ8, page_table, seq_lens, scores,
                                      plan.n_score_cta, status, s, true))) != SA_OK)
     return st;
-  if ((st = cuda_status(launch_select(*g, q, nullptr, nullptr, 0, page_table, seq_lens, scores,
-                                      plan.K, sink / g->P, window / g->P, sel, cnt, phys, status,
-                                      s))) != SA_OK)
+  if ((st = cuda_status(launch_select(*g, page_table, seq_lens, scores, plan.K, sink / g->P,
+                                      window / g->P, sel, cnt, phys, status, s))) != SA_OK)
     return st;
   return run_attend(*g, plan, w, q, k_cache, v_cache, page_table, seq_lens, sel, cnt, phys,
                     plan.K, scale, out, lse, s);

@@ -40,9 +40,9 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
 // fp8: summ holds fp8 records (2 * Dk + 16 bytes per page and KV head)
 cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
                          const int32_t* page_table, const int32_t* seq_lens, float* scores,
-                         int n_cta, int32_t* status, cudaStream_t stream, bool fp8 = false);
-cudaError_t launch_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
-                          int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+                         int n_cta, int32_t* status, cudaStream_t stream, bool fp8 = false,
+                         const void* k_cache = nullptr, int n_tail = 0);
+cudaError_t launch_select(const sa_geom& g, const int32_t* page_table, const int32_t* seq_lens,
                           float* scores, int K, int sink_pages, int window_pages, int32_t* sel,
                           int32_t* sel_count, int32_t* sel_phys, int32_t* status,
                           cudaStream_t stream);

@@ -14,11 +14,14 @@
 // bf16 x bf16 product is exact in fp32; accumulation is fp32.  The G <= 8 query heads
 // are the N=8 side of an m16n8k16 tensor-core tile and 16 pages its M side.
 // The work is a flattened list of tiles (sequence, head group, 16 consecutive pages);
-// each persistent CTA takes a contiguous slice.  A producer warp gathers each tile
-// through the page table with one bulk copy per page (the page's summaries of the
-// head group are contiguous) plus one for the group's query rows, into a ring of
-// shared-memory stages; consumer warps (one per KV head of the group) read A and B
-// fragments with 16-byte shared loads in a permuted channel order (the query side uses
+// each persistent CTA takes a contiguous slice, which every warp derives from the
+// sequence lengths itself (no CTA barrier before the first copy).  A producer warp
+// gathers the slice's page-table entries with asynchronous 4-byte copies, then each
+// tile with one bulk copy per page (the page's summaries of the head group are
+// contiguous, 4 KB for 8 heads at Dk = 128; L2 evict-first) plus one for the group's
+// query rows, into a ring of shared-memory stages; per-tile tables travel with the
+// stage barrier (release/acquire).  Consumer warps (one per KV head of the group) read
+// A and B fragments with 16-byte shared loads in a permuted channel order (the query side uses
 // the same order, so the sum is unchanged) -- page slots are padded by 64 bytes so
 // those loads are free of bank conflicts -- and write the GQA-max score row.
 // HBM-bound: bytes per (page, KV head) = 2 * Dk * 2 (summary) + 4 / Hkv (page table).
@@ -28,11 +31,13 @@
 // to the GQA-max score (a positive power of two commutes with the max).  Bytes per
 // (page, KV head): 2 * Dk + 16.
 //
+// Decode-time refresh: when asked, the consumer warps first recompute the summaries of
+// each sequence's newest pages from K (the pages that received appended tokens) and
+// score them, while the first copies are in flight; the stream skips those pages, so it
+// may read either version of their summaries.
+//
 // Selection (select_kernel, one CTA per (sequence, KV head), launched programmatically
-// dependent on the scoring grid).  Before waiting for the scores it recomputes the
-// summaries of the sequence's newest pages from K when asked (the pages that received
-// appended tokens) and scores them; those scores replace the streamed ones, so the
-// scoring grid may read either version of those summaries.  Then it turns the scores
+// dependent on the scoring grid, which exits before it starts).  It turns the scores
 // into order-preserving 32-bit keys in shared memory (forced pages get key 0, below
 // every real score) and runs an MSB-first radix select with 11-bit digits, starting at
 // the highest bit in which the candidates' keys differ (shared-memory histogram, block
@@ -66,6 +71,9 @@ struct ScoreArgs {
   const int32_t* seq_lens;
   float* scores;  // [B][Hkv][max_pages]
   int32_t* status;
+  const uint4* k_cache;  // bf16 summaries: refresh the newest n_tail pages from K first
+  uint4* summ_w;         // the summaries, written by that refresh
+  int n_tail;
   int B, Hq, Hkv, G, P, max_pages, n_pool;
   int HG, n_hg, WPS, NST;              // heads per tile, head groups, warp groups, stages
   int slot_bytes, q_off, stage_bytes;  // stage: [16][slot_bytes] page slots | q rows
@@ -85,10 +93,6 @@ __device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_
   hi = *reinterpret_cast<const uint32_t*>(&bb);
 }
 
-__device__ __forceinline__ void named_barrier_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // the sequence owning flattened tile u: largest b with pre[b] <= u
 __device__ __forceinline__ int find_seq(const int* pre, int n, int u) {
   int lo = 0, hi = n - 1;
@@ -100,6 +104,37 @@ __device__ __forceinline__ int find_seq(const int* pre, int n, int u) {
       hi = mid - 1;
   }
   return lo;
+}
+
+// Tiles per sequence (n_hg * ceil(pages / 16)) prefix-summed over the batch by one warp;
+// returns the total.  With pre/nbs non-null the prefix and page counts are stored.
+__device__ __forceinline__ int tile_prefix(const ScoreArgs& a, int lane, int* pre, int* nbs) {
+  int carry = 0;
+  for (int b0 = 0; b0 < a.B; b0 += 32) {
+    const int b = b0 + lane;
+    int n = 0;
+    if (b < a.B) {
+      const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
+      const int nb = (L + a.P - 1) / a.P;
+      n = a.n_hg * ((nb + kTilePages - 1) / kTilePages);
+      if (nbs) nbs[b] = nb;
+    }
+    int incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (pre && b < a.B) pre[b] = carry + incl - n;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (pre && lane == 0) pre[a.B] = carry;
+  return carry;
+}
+
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
 }
 
 template <int D, bool F8 = false>
@@ -118,7 +153,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
   int* t_vm = t_np + kMaxTilesPerCta;  // mask of pages with a valid slot
   __shared__ __align__(8) uint64_t full_bar[8];
   __shared__ __align__(8) uint64_t empty_bar[8];
-  __shared__ int sh_nt, abort_flag;
+  __shared__ int abort_flag;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, n_cta = gridDim.x;
 
@@ -132,91 +167,50 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
   }
   // everything read below may come from the previous kernel of the stream: one thread
   // waits for it (which makes its memory visible to this grid), the rest block on the
-  // CTA barrier
+  // CTA barrier.  No early launch of the next grid: the selection grid would start while
+  // most SMs still stream, and its CTAs would pile onto the first SMs to free up (several
+  // per SM, contending); launched as this grid exits, they spread over idle SMs.
   if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
-  asm volatile("griddepcontrol.launch_dependents;");
 
-  if (warp == kScoreConsumers) {
-    // ===================== producer warp: tables =====================
-    // 1. tiles per sequence: n_hg * ceil(pages / 16), prefix-summed
-    int carry = 0;
-    for (int b0 = 0; b0 < a.B; b0 += 32) {
-      const int b = b0 + lane;
-      int n = 0;
-      if (b < a.B) {
-        const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
-        const int nb = (L + a.P - 1) / a.P;
-        n = a.n_hg * ((nb + kTilePages - 1) / kTilePages);
-        nbs[b] = nb;
-      }
-      int incl = n;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      if (b < a.B) pre[b] = carry + incl - n;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) pre[a.B] = carry;
+  // The slice of the flattened tile list this CTA streams: every warp derives it from
+  // the sequence lengths itself, so no CTA-wide barrier stands before the first copy.
+  // Per-tile tables are written by the producer before it arrives on the tile's stage
+  // barrier (release), and read by the consumers after waiting on it (acquire).
+  const bool is_prod = warp == kScoreConsumers;
+  const int total = tile_prefix(a, lane, is_prod ? pre : nullptr, is_prod ? nbs : nullptr);
+  const int W = max(1, (total + n_cta - 1) / n_cta);
+  const int T0 = min(total, c * W);
+  const int nt = min(total, T0 + W) - T0;  // <= kMaxTilesPerCta (the host sizes the grid)
+
+  if (is_prod) {
+    // ===================== producer warp =====================
     __syncwarp();
-    const int total = carry;
-    const int W = max(1, (total + n_cta - 1) / n_cta);
-    const int T0 = min(total, c * W);
-    const int nt = min(total, T0 + W) - T0;  // <= kMaxTilesPerCta (the host sizes the grid)
-    // 2. the slice's tiles: sequence, head group, first page, page count
+    // 1. per tile of the slice (one lane each): sequence, head group, first page, page
+    //    count; its page-table entries gathered by asynchronous 4-byte copies, all in
+    //    flight together
     for (int i = lane; i < nt; i += 32) {
       const int u = T0 + i;
       const int b = find_seq(pre, a.B, u);
       const int ntb = (pre[b + 1] - pre[b]) / a.n_hg;  // tiles per head group
       const int rem = u - pre[b];
-      const int nb = nbs[b];
+      const int p0 = (rem % ntb) * kTilePages;
+      const int np = min(kTilePages, nbs[b] - p0);
       t_b[i] = b;
       t_hg[i] = rem / ntb;
-      t_p0[i] = (rem % ntb) * kTilePages;
-      t_np[i] = min(kTilePages, nb - (rem % ntb) * kTilePages);
+      t_p0[i] = p0;
+      t_np[i] = np;
+      const int32_t* src = a.page_table + (size_t)b * a.max_pages + p0;
+      for (int pg = 0; pg < np; ++pg) cp_async4(ptab + i * kTilePages + pg, src + pg);
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
     __syncwarp();
-    // 3. page-table entries of the slice (16 loads in flight per lane)
-    const int ne = nt * kTilePages;
-    for (int e0 = 0; e0 < ne; e0 += 32 * 16) {
-      int v[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int e = e0 + 32 * k + lane;
-        v[k] = -1;
-        if (e < ne) {
-          const int i = e >> 4, pg = e & 15;
-          if (pg < t_np[i]) v[k] = a.page_table[(size_t)t_b[i] * a.max_pages + t_p0[i] + pg];
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int e = e0 + 32 * k + lane;
-        if (e < ne) ptab[e] = v[k];
-      }
-    }
-    __syncwarp();
-    for (int i = lane; i < nt; i += 32) {
-      int vm = 0;
-      for (int pg = 0; pg < t_np[i]; ++pg) {
-        const int ph = ptab[i * kTilePages + pg];
-        if (ph >= 0 && ph < a.n_pool)
-          vm |= 1 << pg;
-        else
-          report(a.status, SA_ERR_DEVICE_CHECK);
-      }
-      t_vm[i] = vm;
-    }
-    if (lane == 0) sh_nt = nt;
-    __syncwarp();
-    named_barrier_sync(1, kScoreThreads);  // tables ready
 
-    // ===================== producer warp: bulk-copy issue =====================
+    // 2. bulk-copy issue: lanes 0-15 check and copy one page each, lane 16 the queries
     const uint32_t slot_data = (uint32_t)a.HG * a.rec_bytes;  // one page's records of the group
     const uint32_t q_bytes = (uint32_t)a.HG * a.G * D * 2;
     uint64_t t_idle = 0;
+    const uint64_t ef = l2_evict_first();
     for (int k = 0; k < nt;) {
       const int s = k % a.NST;
       bool ready = k < a.NST;
@@ -236,15 +230,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
         continue;
       }
       t_idle = 0;
-      const int vm = t_vm[k], b = t_b[k], hg = t_hg[k];
+      const int b = t_b[k], hg = t_hg[k], np = t_np[k];
+      const int ph = lane < np ? ptab[k * kTilePages + lane] : -1;
+      const bool ok = ph >= 0 && ph < a.n_pool;
+      if (lane < np && !ok) report(a.status, SA_ERR_DEVICE_CHECK);
+      const int vm = (int)(__ballot_sync(0xffffffffu, ok) & 0xFFFFu);
       uint8_t* st = stages + (size_t)s * a.stage_bytes;
-      if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], __popc(vm) * slot_data + q_bytes);
+      if (lane == 0) {
+        t_vm[k] = vm;
+        mbar_arrive_expect_tx(&full_bar[s], __popc(vm) * slot_data + q_bytes);
+      }
       __syncwarp();
-      if (lane < kTilePages && ((vm >> lane) & 1)) {
-        const int ph = ptab[k * kTilePages + lane];
-        bulk_load(st + lane * a.slot_bytes,
-                  a.summ + ((size_t)ph * a.Hkv + hg * a.HG) * (size_t)a.rec_bytes, slot_data,
-                  &full_bar[s]);
+      if (ok) {
+        bulk_load_hint(st + lane * a.slot_bytes,
+                       a.summ + ((size_t)ph * a.Hkv + hg * a.HG) * (size_t)a.rec_bytes,
+                       slot_data, &full_bar[s], ef);
       } else if (lane == kTilePages) {
         bulk_load(st + a.q_off, a.q + ((size_t)b * a.Hq + (size_t)hg * a.HG * a.G) * D, q_bytes,
                   &full_bar[s]);
@@ -253,10 +253,29 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
     }
   } else {
     // ===================== consumer warps =====================
-    named_barrier_sync(1, kScoreThreads);  // tables ready
+    // 0. decode-time refresh of the newest pages' summaries from K (the pages that
+    //    received appended tokens), spread over the grid's consumer warps while the first
+    //    copies are in flight.  Their scores replace the streamed ones (the stream skips
+    //    those pages), so the stream may read either version of the summaries.
+    if constexpr (!F8) {
+      const int n_items = a.B * a.Hkv * a.n_tail;
+      for (int i = c + n_cta * warp; i < n_items; i += n_cta * kScoreConsumers) {
+        const int pr = i / a.n_tail;
+        const int b = pr / a.Hkv, h = pr % a.Hkv;
+        const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
+        const int lp = (L + a.P - 1) / a.P - a.n_tail + i % a.n_tail;
+        if (lp < 0) continue;
+        const int ph = a.page_table[(size_t)b * a.max_pages + lp];
+        float sc = 0.f;
+        if (ph >= 0 && ph < a.n_pool)
+          sc = warp_refresh_and_score<D>(a.k_cache, a.summ_w,
+                                         a.q + ((size_t)b * a.Hq + h * a.G) * D, a.G, ph, h,
+                                         a.Hkv, a.P, min(a.P, L - lp * a.P), lane);
+        if (lane == 0) a.scores[(size_t)pr * a.max_pages + lp] = sc;
+      }
+    }
     const int r = lane >> 2, t = lane & 3;
     const int grp = warp / a.HG, hh = warp % a.HG;  // stage group, head within the group
-    const int nt = sh_nt;
     const bool v0 = 2 * t < a.G, v1 = 2 * t + 1 < a.G;
     for (int k = grp; k < nt; k += a.WPS) {
       const int s = k % a.NST;
@@ -321,9 +340,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
           m1 = ldexpf(m1, (int)(int8_t)sp[(r + 8) * a.slot_bytes]);
         }
         if (t == 0) {
+          // pages refreshed above keep the score computed from their fresh summary
+          const int lim = a.n_tail > 0 ? min(np, nbs[b] - a.n_tail - p0) : np;
           float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages + p0;
-          if (r < np) srow[r] = m0;
-          if (r + 8 < np) srow[r + 8] = m1;
+          if (r < lim) srow[r] = m0;
+          if (r + 8 < lim) srow[r + 8] = m1;
         }
       }
       __syncwarp();
@@ -349,9 +370,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
 }
 
 struct SelectArgs {
-  const uint16_t* q;
-  uint4* summ;
-  const uint4* k_cache;  // non-null: refresh the newest n_tail pages' summaries first
   const int32_t* page_table;
   const int32_t* seq_lens;
   float* scores;       // [B][Hkv][max_pages]
@@ -359,11 +377,10 @@ struct SelectArgs {
   int32_t* sel_count;  // [B][Hkv]
   int32_t* sel_phys;   // [B][Hkv][K] physical pages of the selection (nullable)
   int32_t* status;
-  int Hq, Hkv, P, max_pages, n_pool, K, s_pages, w_pages, n_tail;
+  int Hkv, P, max_pages, K, s_pages, w_pages;
   int ptab_in_smem;  // the sequence's page-table row is staged next to the keys
 };
 
-template <int D>
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs a) {
   constexpr int NT = kSelectThreads;
   using Bar = SelBar<-1, NT>;
@@ -373,40 +390,22 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
   __shared__ uint32_t bin_key[kBinCap];
   __shared__ int bin_page[kBinCap];
   __shared__ int warp_tot[NT / 32 + 1];
-  __shared__ float tail_score[kMaxTail];
   const SelScratch sh{hist, bin_key, bin_page, warp_tot, red, misc};
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x, b = blockIdx.y;
-  const int G = a.Hq / a.Hkv;
   // The scoring grid passed its own wait before letting this grid start, so the
   // inputs of the call (everything but the scores) are complete here.
   const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
   const int nb = (L + a.P - 1) / a.P;
   const int32_t* ptab_g = a.page_table + (size_t)b * a.max_pages;
   float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages;
-  const int tail0 = max(0, nb - a.n_tail);
-  const int n_tail = a.k_cache ? nb - tail0 : 0;
-  // 1. decode-time refresh of the newest pages (overlaps the scoring grid).  The latent
-  //    geometry refreshes in a kernel of its own before scoring (k_cache is null here).
-  if constexpr (D <= 128) {
-    for (int i = warp; i < n_tail; i += NT / 32) {
-      const int lp = tail0 + i;
-      const int ph = ptab_g[lp];
-      float sc = 0.f;
-      if (ph >= 0 && ph < a.n_pool)
-        sc = warp_refresh_and_score<D>(a.k_cache, a.summ, a.q + ((size_t)b * a.Hq + h * G) * D,
-                                       G, ph, h, a.Hkv, a.P, min(a.P, L - lp * a.P), lane);
-      if (lane == 0) tail_score[i] = sc;
-    }
-  }
-  // 2. wait for the scores (one thread; the rest block on the CTA barrier)
+  // 1. wait for the scores (one thread; the rest block on the CTA barrier)
   if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;");
   int32_t* out = a.sel + ((size_t)b * a.Hkv + h) * a.K;
   int32_t* cnt_out = a.sel_count + (size_t)b * a.Hkv + h;
   int32_t* phys_out = a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.K : nullptr;
-  for (int i = tid; i < n_tail; i += NT) srow[tail0 + i] = tail_score[i];
   const int K = a.K;
   if (nb <= K) {  // everything fits the budget
     for (int i = tid; i < K; i += NT) {
@@ -417,7 +416,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
     return;
   }
   int32_t* ptab_s = a.ptab_in_smem ? reinterpret_cast<int32_t*>(keys + a.max_pages) : nullptr;
-  // 3. keys (8 loads in flight per thread) and the candidates' key range
+  // 2. keys (8 loads in flight per thread) and the candidates' key range
   const int wbeg = nb - a.w_pages;
   uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
   for (int p0 = 0; p0 < nb; p0 += NT * 8) {
@@ -433,7 +432,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
     for (int k = 0; k < 8; ++k) {
       const int p = p0 + k * NT + tid;
       if (p < nb) {
-        const float sv = (n_tail > 0 && p >= tail0) ? tail_score[p - tail0] : v[k];
+        const float sv = v[k];
         const bool forced = p < a.s_pages || p >= wbeg;
         const uint32_t key = forced ? 0u : f32_order_key(sv);
         keys[p] = key;
@@ -447,11 +446,11 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
   }
   block_key_range<NT, Bar>(kmn, kmx, red);
 
-  // 4. threshold: a candidate is taken when its key >= thr or it was marked kWin
+  // 3. threshold: a candidate is taken when its key >= thr or it was marked kWin
   const uint64_t thr = radix_select_threshold<NT, Bar>(keys, nb, a.s_pages, wbeg,
                                                        K - a.s_pages - a.w_pages, kmn, kmx, sh);
 
-  // 5. ascending list: forced pages and taken candidates.  Each warp owns a contiguous
+  // 4. ascending list: forced pages and taken candidates.  Each warp owns a contiguous
   // run of pages (a multiple of 32) and compacts it with ballots; one block barrier
   // gives every warp its offset.
   auto taken = [&](int p) {
@@ -608,14 +607,23 @@ static ScoreArgs make_score_args(const sa_geom& g, const void* q, const void* su
   a.P = g.P;
   a.max_pages = g.max_pages;
   a.n_pool = g.n_pool;
+  a.k_cache = nullptr;
+  a.summ_w = nullptr;
+  a.n_tail = 0;
   score_shape(g, &a, f8);
   return a;
 }
 
 cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
                          const int32_t* page_table, const int32_t* seq_lens, float* scores,
-                         int n_cta, int32_t* status, cudaStream_t stream, bool fp8) {
+                         int n_cta, int32_t* status, cudaStream_t stream, bool fp8,
+                         const void* k_cache, int n_tail) {
   ScoreArgs a = make_score_args(g, q, summ, page_table, seq_lens, scores, status, fp8);
+  if (!fp8 && k_cache && n_tail > 0) {
+    a.k_cache = static_cast<const uint4*>(k_cache);
+    a.summ_w = static_cast<uint4*>(const_cast<void*>(summ));
+    a.n_tail = n_tail < kMaxTail ? n_tail : kMaxTail;
+  }
   const size_t smem = score_smem(g, a);
   const void* kern;
   if (g.Dk == 64)
@@ -637,24 +645,12 @@ cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
   return launch_pdl(kern, dim3(n_cta), dim3(kScoreThreads), smem, stream, args);
 }
 
-cudaError_t launch_select(const sa_geom& g, const void* q, void* summ, const void* k_cache,
-                          int n_tail, const int32_t* page_table, const int32_t* seq_lens,
+cudaError_t launch_select(const sa_geom& g, const int32_t* page_table, const int32_t* seq_lens,
                           float* scores, int K, int sink_pages, int window_pages, int32_t* sel,
                           int32_t* sel_count, int32_t* sel_phys, int32_t* status,
                           cudaStream_t stream) {
-  const void* skern;
-  if (g.Dk == 64)
-    skern = reinterpret_cast<const void*>(select_kernel<64>);
-  else if (g.Dk == 128)
-    skern = reinterpret_cast<const void*>(select_kernel<128>);
-  else if (g.Dk == 576 && n_tail == 0)
-    skern = reinterpret_cast<const void*>(select_kernel<576>);
-  else
-    return cudaErrorInvalidValue;
+  const void* skern = reinterpret_cast<const void*>(select_kernel);
   SelectArgs s;
-  s.q = static_cast<const uint16_t*>(q);
-  s.summ = static_cast<uint4*>(summ);
-  s.k_cache = n_tail > 0 ? static_cast<const uint4*>(k_cache) : nullptr;
   s.page_table = page_table;
   s.seq_lens = seq_lens;
   s.scores = scores;
@@ -662,15 +658,12 @@ cudaError_t launch_select(const sa_geom& g, const void* q, void* summ, const voi
   s.sel_count = sel_count;
   s.sel_phys = sel_phys;
   s.status = status;
-  s.Hq = g.Hq;
   s.Hkv = g.Hkv;
   s.P = g.P;
   s.max_pages = g.max_pages;
-  s.n_pool = g.n_pool;
   s.K = K;
   s.s_pages = sink_pages;
   s.w_pages = window_pages;
-  s.n_tail = n_tail < kMaxTail ? n_tail : kMaxTail;
   const size_t keys_bytes = (size_t)g.max_pages * 4;
   s.ptab_in_smem = 2 * keys_bytes <= (size_t)200 * 1024;
   const size_t ssmem = s.ptab_in_smem ? 2 * keys_bytes : keys_bytes;
@@ -688,11 +681,12 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
                                 float* scores, int n_cta, int K, int sink_pages,
                                 int window_pages, int32_t* sel, int32_t* sel_count,
                                 int32_t* sel_phys, int32_t* status, cudaStream_t stream) {
-  cudaError_t e =
-      launch_score(g, q, summ, page_table, seq_lens, scores, n_cta, status, stream);
+  // the newest pages' refresh runs inside the scoring grid
+  cudaError_t e = launch_score(g, q, summ, page_table, seq_lens, scores, n_cta, status, stream,
+                               false, k_cache, n_tail);
   if (e != cudaSuccess) return e;
-  return launch_select(g, q, summ, k_cache, n_tail, page_table, seq_lens, scores, K, sink_pages,
-                       window_pages, sel, sel_count, sel_phys, status, stream);
+  return launch_select(g, page_table, seq_lens, scores, K, sink_pages, window_pages, sel,
+                       sel_count, sel_phys, status, stream);
 }
 
 }  // namespace sa
