@@ -61,7 +61,7 @@ constexpr int kScoreConsumers = 8;
 constexpr int kScoreThreads = (kScoreConsumers + 1) * 32;
 constexpr int kMaxTilesPerCta = 64;
 constexpr int kSlotPad = 64;  // odd multiple of 64 B between page slots: no bank conflicts
-constexpr int kSelectThreads = 256;
+constexpr int kSelectThreads = 512;
 constexpr int kScoreSmemLimit = 227 * 1024;
 
 struct ScoreArgs {
