@@ -3,12 +3,18 @@
 One step = one decode step of a 32-layer model with Llama-3.1-8B attention geometry
 (batch 8, 32 query / 8 KV heads, head dim 128, 32768 tokens per sequence, page 16,
 token budget 2048 = sink 64 + window 512 + top-k).  Per layer, one sa_sparse_decode call
-scores every page against the query (streaming kernel), selects the top pages (per-pair
-select kernel, which also refreshes the summary of each sequence's newest page) and runs
-split-KV attention over the gathered pages
-(attention kernel plus the merge kernel of the pairs split across warps).  Its two
-halves, sa_select_pages and sa_attend_selected, are timed apart for context.  Every layer owns its own KV pool, so a step touches ~4.3 GB (> L2)
-and nothing is served from L2 across layers.
+scores every page against the query (streaming kernel, which also refreshes the summary
+of each sequence's newest page from K), selects the top pages (per-pair select kernel)
+and runs split-KV attention over the gathered pages (attention kernel plus the merge
+kernel of the pairs split across warps).  Its two halves, sa_select_pages and
+sa_attend_selected, are timed apart for context.  Every layer owns its own KV pool, so a
+step touches ~4.3 GB (> L2) and nothing is served from L2 across layers.
+
+The default llama32k run also times llama128k (131072 tokens per sequence), ragged
+(4 sequences of 64K-256K tokens, page 32) and mla (latent 576/512, 128 query heads) the
+same way over 8 layer pools each and adds their microseconds per layer-call and HBM
+fractions to the line's config (--no-extras skips them).  cpu_baseline is the CPU oracle
+on every host core (independent sequences on threads), its single-thread rate beside it.
 
 Metric: sparse-decode seq*heads/s = (sequence, query head) attention outputs of one
 layer-call per second, whole job.  The headline is timed on a CUDA graph of the step
@@ -58,7 +64,10 @@ def parse():
     ap.add_argument("--layers", type=int, default=None,
                     help="layer pools per step (default 32 for llama32k, 8 otherwise)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="llama32k: skip the llama128k / ragged / mla measurements that the "
+                         "default run adds to the line's config")
     ap.add_argument("--seed", type=int, default=0,
                     help="offset added to the workload's seed (every rank adds its own)")
     ap.add_argument("--summaries", default="bf16", choices=["bf16", "fp8"],
@@ -230,6 +239,56 @@ def oracle_sample(case, seconds, select_every=1, fp8=False):
     return units / t_total, done, t_total
 
 
+def oracle_sample_mt(case, seconds, select_every=1, fp8=False, threads=None):
+    """oracle_sample on `threads` host threads at once (default: every core), each on its
+    own sequences (thread i takes sequences i, i + threads, ...): the C oracle releases
+    the GIL while it computes, so independent sequences run in parallel.  Returns
+    (units per second of wall time, calls done, wall seconds, threads)."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    threads = threads or os.cpu_count() or 1
+    threads = max(1, min(threads, case.geom.B))
+    oracle.load()  # build/load once, before the threads start
+
+    def worker(i):
+        sub = dataclass_slice(case, i, threads)
+        _, done, _ = oracle_sample(sub, seconds, select_every, fp8)
+        return done
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        dones = list(ex.map(worker, range(threads)))
+    wall = time.perf_counter() - t0
+    done = sum(dones)
+    return done * case.geom.Hq / wall, done, wall, threads
+
+
+def dataclass_slice(case, i, step):
+    """The decode case restricted to sequences i, i + step, ... (same pool)."""
+    import dataclasses
+    idx = np.arange(i, case.geom.B, step)
+    g = dataclasses.replace(case.geom, B=len(idx))
+    return dataclasses.replace(case, geom=g, q=case.q[idx], page_table=case.page_table[idx],
+                               seq_lens=case.seq_lens[idx])
+
+
+def workload_config(case, args, layers):
+    """The workload description shared by the native and the reference lines."""
+    g = case.geom
+    fp8 = args.summaries == "fp8"
+    R = args.select_every
+    return {
+        "workload": args.workload,
+        "batch": g.B, "q_heads": g.Hq, "kv_heads": g.Hkv, "head_dim": g.Dk,
+        "seq_len": int(case.seq_lens.max()), "page": g.P, "budget_tokens": case.budget,
+        "sink": case.sink, "window": case.window, "layers_per_step": layers,
+        "select_every": R,
+        "summaries": "fp8 e4m3 rounded outward" if fp8 else "bf16",
+        "call": ("sa_sparse_decode_fp8" if fp8 else "sa_sparse_decode") if R == 1 else
+                "sa_select_pages + sa_attend_selected",
+    }
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -249,21 +308,21 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}, default=_json_default), flush=True)
         return 0
     case = synth.decode_case(args.workload, seed=rank_seed(args.workload, 0, args.seed))
-    v, done, t = oracle_sample(case, args.cpu_seconds, args.select_every,
-                               args.summaries == "fp8")
+    v, done, t, cores = oracle_sample_mt(case, args.cpu_seconds, args.select_every,
+                                         args.summaries == "fp8")
     line = {
         "impl": "reference", "metric": "sparse-decode seq*heads/s", "value": v,
         "unit": "seq*heads/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "ms_per_step": None,
-        "config": {"workload": args.workload, "layers_per_step": args.layers,
-                   "select_every": args.select_every, "summaries": args.summaries},
-        "cpu_baseline": {"value": v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
+        "config": workload_config(case, args, args.layers),
+        "cpu_baseline": {"value": v, "unit": "seq*heads/s", "cores": cores, "kind": "oracle",
                          "sample": "%d (sequence, layer) decode calls of layer 0 "
-                                   "(score+select%s, attend; all %d heads), %.1f s" % (
+                                   "(score+select%s, attend; all %d heads) on %d host "
+                                   "threads, %.1f s wall" % (
                                        done, "" if args.select_every == 1 else
                                        " every %d layers" % args.select_every,
-                                       case.geom.Hq, t)},
+                                       case.geom.Hq, cores, t)},
         "e2e": {"value": v, "unit": "seq*heads/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -510,9 +569,19 @@ def run_native(args, rank, world, dist):
         "score_stream_kernel<fp8>" if F8 else "score_stream_kernel")
     dom_bytes, dom_ms = sel_b, sc_mean
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    cpu_v, cpu_done, cpu_t = (None, 0, 0.0)
+    cpu_v, cpu_done, cpu_t, cpu_cores = (None, 0, 0.0, 0)
+    cpu1 = (None, 0, 0.0)
     if world == 1:
-        cpu_v, cpu_done, cpu_t = oracle_sample(case, args.cpu_seconds, R, F8)
+        cpu_v, cpu_done, cpu_t, cpu_cores = oracle_sample_mt(case, args.cpu_seconds, R, F8)
+        cpu1 = oracle_sample(case, args.cpu_seconds / 2, R, F8)
+    extras = {}
+    if world == 1 and args.extras and args.workload == "llama32k" and R == 1 and not F8:
+        # free the headline's pools first: the other configurations need the room
+        del ks, vs, qs, summs, k0, v0, graph, graph_ev, graph_sc
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        for name in ("llama128k", "ragged", "mla"):
+            extras.update(extra_decode(name, args, dev, hbm_peak))
     # GQA: score, select (+ tail refresh), attention, merge; latent: tail refresh, query
     # sign split, tensor-core score, select, tensor-core attention, merge
     # select half of one layer-call (fp8: the newest pages' records in a kernel of their own)
@@ -533,14 +602,7 @@ def run_native(args, rank, world, dist):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": args.workload,
-            "batch": g.B, "q_heads": g.Hq, "kv_heads": g.Hkv, "head_dim": g.Dk,
-            "seq_len": int(case.seq_lens.max()), "page": P, "budget_tokens": case.budget,
-            "sink": case.sink, "window": case.window, "layers_per_step": L_layers,
-            "select_every": R,
-            "summaries": "fp8 e4m3 rounded outward" if F8 else "bf16",
-            "call": ("sa_sparse_decode_fp8" if F8 else "sa_sparse_decode") if R == 1 else
-                    "sa_select_pages + sa_attend_selected",
+            **workload_config(case, args, L_layers),
             "l2": "inputs larger than L2: %d distinct layer pools, %.2f GB touched per step"
                   % (L_layers, step_bytes / 1e9),
             "parallelism": "replicas (batch split), no collective" if world > 1 else "1 GPU",
@@ -554,6 +616,7 @@ def run_native(args, rank, world, dist):
             "summaries_gbs_alone": summ_bytes / (summ_ms * 1e-3) / 1e9,
             "algorithmic_bytes_per_layer": step_bytes / L_layers,
             **mla_flops(case, sel_count, sc_mean, att_mean),
+            **extras,
         },
         "roofline": {
             "kernel": dom_kernel,
@@ -563,10 +626,13 @@ def run_native(args, rank, world, dist):
             "traffic": recorded_traffic(dom_kernel, args.workload),
         },
         "cpu_baseline": None if cpu_v is None else {
-            "value": cpu_v, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
+            "value": cpu_v, "unit": "seq*heads/s", "cores": cpu_cores, "kind": "oracle",
             "sample": "%d (sequence, layer) decode calls of layer 0 (score+select%s, attend; "
-                      "all %d query heads), %.1f s single-threaded" % (
-                          cpu_done, "" if R == 1 else " every %d layers" % R, g.Hq, cpu_t)},
+                      "all %d query heads) on %d host threads (independent sequences), "
+                      "%.1f s wall" % (cpu_done, "" if R == 1 else " every %d layers" % R,
+                                       g.Hq, cpu_cores, cpu_t),
+            "single_thread_value": cpu1[0],
+            "single_thread_sample": "%d calls, %.1f s on one thread" % (cpu1[1], cpu1[2])},
         "e2e": {"value": whole_job_rate(units_per_step, world, e2e_ms), "unit": "seq*heads/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -574,6 +640,87 @@ def run_native(args, rank, world, dist):
     }
     print(json.dumps(line, default=_json_default), flush=True)
     return 0
+
+
+def extra_decode(name, args, dev, hbm_peak, layers=8, steps=10, warmup=3):
+    """One more decode configuration timed the headline's way (a CUDA graph of `layers`
+    sa_sparse_decode calls over distinct layer pools, inputs resident, CUDA events), for
+    the line's config: microseconds per layer-call and the fraction of HBM peak at the
+    algorithmic bytes; the latent geometry adds its tensor-core rate."""
+    import torch
+    import paged_kv_cache_sa_b200 as sa
+    from paged_kv_cache_sa_b200 import Geometry
+
+    case = synth.decode_case(name, seed=rank_seed(name, 0, args.seed))
+    g = Geometry.of(case.geom)
+    P = g.P
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16
+                                                          else a)).to(dev)
+    k0 = t(case.k_cache)
+    v0 = t(case.v_cache) if case.v_cache is not None else None
+    pt, sl = t(case.page_table), t(case.seq_lens)
+    rng = np.random.default_rng(4321)
+    stride = max(1, g.n_pool // layers)
+    ks, vs, qs, summs = [], [], [], []
+    for l in range(layers):
+        ks.append(k0 if l == 0 else torch.roll(k0, shifts=l * stride, dims=0))
+        vs.append(None if v0 is None else (v0 if l == 0 else torch.roll(v0, shifts=l * stride, dims=0)))
+        qn = case.q if l == 0 else synth.f32_to_bf16(rng.standard_normal(case.q.shape).astype(np.float32))
+        qs.append(t(qn))
+        summs.append(torch.empty((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device=dev))
+        sa.page_summaries(g, ks[l], pt, sl, summs[l])
+    K = case.budget // P
+    ws = sa.Workspace.for_decode(g, case.budget)
+    sel = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((g.B, g.Hkv), dtype=torch.int32, device=dev)
+    out = torch.empty((g.B, g.Hq, g.Dv), dtype=torch.float32, device=dev)
+    lse = torch.empty((g.B, g.Hq), dtype=torch.float32, device=dev)
+
+    def run():
+        for l in range(layers):
+            sa.sparse_decode(g, qs[l], ks[l], vs[l], summs[l], pt, sl, case.budget, case.sink,
+                             case.window, case.scale, ws, out=out, lse=lse, sel_out=sel,
+                             sel_count_out=cnt, n_tail_refresh=1)
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    assert ws.status() == sa.SA_OK
+    sel_count = cnt.cpu().numpy()
+    sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, P)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    assert ws.status() == sa.SA_OK
+    us = e0.elapsed_time(e1) * 1e3 / (steps * layers)
+    layer_b = sel_b + att_b + upd_b
+    res = {
+        name + "_us_per_layer": us,
+        name + "_algorithmic_bytes_per_layer": layer_b,
+        name + "_frac_of_hbm_peak": layer_b / (us * 1e-6) / 1e9 / hbm_peak,
+        name + "_layers_timed": layers,
+    }
+    if g.v_aliases_k:
+        fl = mla_flops(case, sel_count, 1.0, 1.0)
+        tot = (fl["score_gflop_per_layer"] + fl["attend_gflop_per_layer"]) * 1e9
+        res[name + "_tensor_tflops"] = tot / (us * 1e-6) / 1e12
+    del graph, ks, vs, qs, summs, k0, v0
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
 
 
 def mla_flops(case, sel_count, score_ms, attend_ms):

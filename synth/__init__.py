@@ -9,7 +9,9 @@ arithmetic (no summaries, scores, selection, attention or compaction); both the
 CPU oracle and the CUDA path consume what it returns.
 
 Random numbers come from numpy's PCG64 seeded through ``SeedSequence([seed,
-stream])``, one stream per tensor, and are rounded to bf16 with
+stream])``, one stream per tensor (``SeedSequence([seed, stream, chunk])`` per block
+of 2^22 values for the large normal tensors, so that the blocks can be drawn on
+several host threads with the same result), and are rounded to bf16 with
 round-to-nearest-even.  bf16 tensors are returned as ``uint16`` bit patterns.
 
 Workloads (sizes as named by the method's target configurations):
@@ -39,6 +41,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
 from typing import Optional
 
 import numpy as np
@@ -79,17 +82,35 @@ def _rng(seed: int, stream: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), int(stream)])))
 
 
-def _normal_bf16(rng: np.random.Generator, shape, sigma: float = 1.0,
-                 chunk: int = 1 << 24) -> np.ndarray:
-    """N(0, sigma^2) samples rounded to bf16, generated in chunks to bound memory."""
+_CHUNK = 1 << 22
+
+
+def _normal_bf16(seed: int, stream: int, shape, sigma: float = 1.0) -> np.ndarray:
+    """N(0, sigma^2) samples rounded to bf16.  Block c of 2^22 values comes from its own
+    stream SeedSequence([seed, stream, c]); blocks are drawn on host threads (numpy
+    releases the GIL while filling), the result does not depend on the thread count."""
+    from concurrent.futures import ThreadPoolExecutor
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        x = rng.standard_normal(e - s, dtype=np.float32)
+
+    def block(c: int) -> None:
+        s0 = c * _CHUNK
+        e = min(n, s0 + _CHUNK)
+        rng = np.random.Generator(np.random.PCG64(
+            np.random.SeedSequence([int(seed), int(stream), c])))
+        x = rng.standard_normal(e - s0, dtype=np.float32)
         if sigma != 1.0:
             x *= np.float32(sigma)
-        out[s:e] = f32_to_bf16(x)
+        out[s0:e] = f32_to_bf16(x)
+
+    n_blocks = (n + _CHUNK - 1) // _CHUNK
+    workers = max(1, min(16, os.cpu_count() or 1, n_blocks))
+    if workers == 1:
+        for c in range(n_blocks):
+            block(c)
+    else:
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(block, range(n_blocks)))
     return out.reshape(shape)
 
 
@@ -232,9 +253,9 @@ def decode_case(workload: str, *, seed: Optional[int] = None, B: Optional[int] =
         page_table[b, :nb] = phys[o:o + nb]
         o += nb
 
-    q = _normal_bf16(_rng(seed_, _S_Q), (Bn, Hq_, Dk_))
-    k_cache = _normal_bf16(_rng(seed_, _S_K), (n_pool, Hkv_, Pn, Dk_), w["sigma"])
-    v_cache = None if w["mla"] else _normal_bf16(_rng(seed_, _S_V), (n_pool, Hkv_, Pn, Dv_),
+    q = _normal_bf16(seed_, _S_Q, (Bn, Hq_, Dk_))
+    k_cache = _normal_bf16(seed_, _S_K, (n_pool, Hkv_, Pn, Dk_), w["sigma"])
+    v_cache = None if w["mla"] else _normal_bf16(seed_, _S_V, (n_pool, Hkv_, Pn, Dv_),
                                                  w["sigma"])
 
     if w["outliers"]:
@@ -359,14 +380,13 @@ def prune_case(workload: str = "prune", *, extra_free: int = 0, keep_all: bool =
         need += (int(keep[b, :L].sum()) + P - 1) // P
     n_free = need + int(extra_free)
     # grow the pool by n_free fresh pages (filled with seeded noise)
-    rng = _rng(base.seed, 100)
-    k_new = _normal_bf16(rng, (n_free,) + base.k_cache.shape[1:])
+    k_new = _normal_bf16(base.seed, 100, (n_free,) + base.k_cache.shape[1:])
     k_cache = np.concatenate([base.k_cache, k_new], axis=0)
     v_cache = None
     if base.v_cache is not None:
-        v_new = _normal_bf16(rng, (n_free,) + base.v_cache.shape[1:])
+        v_new = _normal_bf16(base.seed, 101, (n_free,) + base.v_cache.shape[1:])
         v_cache = np.concatenate([base.v_cache, v_new], axis=0)
-    free_pages = (g.n_pool + rng.permutation(n_free)).astype(np.int32)
+    free_pages = (g.n_pool + _rng(base.seed, 102).permutation(n_free)).astype(np.int32)
     geom = dataclasses.replace(g, n_pool=g.n_pool + n_free)
     dec = dataclasses.replace(base, geom=geom, k_cache=k_cache, v_cache=v_cache)
     return PruneCase(dec, keep, free_pages)
