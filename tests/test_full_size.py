@@ -85,3 +85,34 @@ def test_full_size_bench_launch_config(wl):
         assert np.array_equal(u16(dc.summ), summ)
         assert np.array_equal(out2.cpu().numpy(), out.cpu().numpy())
         assert np.array_equal(lse2.cpu().numpy(), lse.cpu().numpy())
+
+
+def test_prune_full_size_bench_config():
+    """Prefix-cache pruning compaction at the size bench.py times (SparseEngine blog,
+    Prefix-Cache Pruning paragraph): 32 sessions of 8K-64K tokens, page 16, 8 KV heads,
+    keep-mask of sink + window + random spans.  Every output bit-exact: new page table,
+    lengths, position map, logical lengths, the whole K/V pool and the new pages'
+    summaries."""
+    import torch
+    import paged_kv_cache_sa_b200 as sa
+    pc = synth.prune_case("prune")
+    d = pc.decode
+    g = sa.Geometry.of(d.geom)
+    assert g.B == 32
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(
+        a.view(np.int16) if a.dtype == np.uint16 else a)).cuda()
+    k, v = to_dev(d.k_cache), to_dev(d.v_cache)
+    summ = torch.zeros((g.n_pool, g.Hkv, 2, g.Dk), dtype=torch.int16, device="cuda")
+    ws = sa.Workspace.for_prune(g)
+    npt, nsl, pos, ll = sa.prune_compact(g, k, v, to_dev(d.page_table), to_dev(d.seq_lens),
+                                         to_dev(pc.keep), to_dev(pc.free_pages), k, v, summ, ws)
+    assert ws.status() == sa.SA_OK
+    ref = oracle.prune_compact(d.geom, d.k_cache, d.v_cache, d.page_table, d.seq_lens, pc.keep,
+                               pc.free_pages)
+    assert np.array_equal(npt.cpu().numpy(), ref["new_page_table"])
+    assert np.array_equal(nsl.cpu().numpy(), ref["new_seq_lens"])
+    assert np.array_equal(pos.cpu().numpy(), ref["pos_map"])
+    assert np.array_equal(ll.cpu().numpy(), ref["logical_len"])
+    assert np.array_equal(u16(k), ref["k_dst"])
+    assert np.array_equal(u16(v), ref["v_dst"])
+    assert np.array_equal(u16(summ), ref["summ"])

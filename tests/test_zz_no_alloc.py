@@ -8,8 +8,9 @@ and geometries whose workspace exceeds the scratch are refused before any launch
 import numpy as np
 import pytest
 
+import oracle
 import synth
-from parity import DevCase, check_attention
+from parity import DevCase, check_attention, check_selection
 
 pytestmark = pytest.mark.gpu
 
@@ -22,13 +23,16 @@ import paged_kv_cache_sa_b200 as sa  # noqa: E402
 
 @pytest.mark.parametrize("kw", [dict(wl="llama32k", B=2, L=(8192, 8192), seed=81),
                                 dict(wl="tiny", B=3, seq_lens=[4096, 700, 0], Hkv=2, Hq=8,
-                                     seed=82)])
+                                     seed=82),
+                                # latent geometry small enough for the static scratch
+                                dict(wl="mla", B=2, L=(8192, 8192), seed=83)])
 def test_noalloc_matches_workspace_decode_on_consecutive_calls(kw):
     kw = dict(kw)
     case = synth.decode_case(kw.pop("wl"), **kw)
     dc = DevCase(case)
     g = dc.g
     K = case.budget // g.P
+    assert sa.decode_workspace_size(g, case.budget) <= 32 << 20
     sa.page_summaries(g, dc.k, dc.pt, dc.sl, dc.summ)
     ws = sa.Workspace.for_decode(g, case.budget)
     sel_r = torch.empty((g.B, g.Hkv, K), dtype=torch.int32, device="cuda")
@@ -51,6 +55,13 @@ def test_noalloc_matches_workspace_decode_on_consecutive_calls(kw):
         assert np.array_equal(sel.cpu().numpy(), ref[2])
         assert np.array_equal(cnt.cpu().numpy(), ref[3])
         check_attention(out.cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
+    # and against the oracle: the selection bit-exact outside the tie band, the attention
+    # over the selection made within the stated tolerance
+    o = oracle.decode(case)
+    check_selection(case.geom, case.seq_lens, case.budget, case.sink, case.window,
+                    o["scores"], o["sel"], o["sel_count"], ref[2], ref[3])
+    oa = oracle.decode(case, sel=ref[2], sel_count=ref[3])
+    check_attention(out.cpu().numpy(), lse.cpu().numpy(), oa["out"], oa["lse"])
 
 
 def test_noalloc_refuses_workspace_above_the_scratch():
