@@ -670,41 +670,47 @@ __global__ void __launch_bounds__(mla::kAttnThreads, 1) attend_mla_kernel(const 
 
 // Combine the chunk states of each (sequence, head): out = sum_s 2^(m_s - M) O_s / L,
 // lse = (M + log2 L) ln 2.  CTA = (sequence, 32 channels); thread = head.
+constexpr int kMergeCh = 8;  // channels per merge CTA: B * 64 CTAs at the latent geometry
+
 __global__ void __launch_bounds__(128) attend_mla_merge_kernel(const float* __restrict__ part_o,
                                                                const float* __restrict__ part_ml,
                                                                float* __restrict__ out,
                                                                float* __restrict__ lse,
                                                                int n_split) {
   using namespace mla;
-  __shared__ float tile[kG][33];
+  __shared__ float tile[kG][kMergeCh + 1];
   if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;");
-  const int b = blockIdx.y, c0 = blockIdx.x * 32, h = threadIdx.x;
+  const int b = blockIdx.y, c0 = blockIdx.x * kMergeCh, h = threadIdx.x;
   const float* ml = part_ml + (size_t)b * n_split * kG * 2;
+  // running maximum first (the splits' loads in flight together), then the weighted
+  // sums in split order
   float M = -INFINITY;
+#pragma unroll 8
   for (int s = 0; s < n_split; ++s) M = fmaxf(M, ml[((size_t)s * kG + h) * 2]);
-  float Lsum = 0.f, acc[32];
+  float Lsum = 0.f, acc[kMergeCh];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+  for (int i = 0; i < kMergeCh; ++i) acc[i] = 0.f;
+#pragma unroll 4
   for (int s = 0; s < n_split; ++s) {
     const float ms = ml[((size_t)s * kG + h) * 2];
-    if (ms == -INFINITY) continue;
+    if (ms == -INFINITY) continue;  // an empty chunk: its O is not read
     const float w = fast_exp2(ms - M);
     Lsum += w * ml[((size_t)s * kG + h) * 2 + 1];
     const float* po = part_o + (((size_t)b * n_split + s) * kDv + c0) * kG + h;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] += w * po[(size_t)i * kG];
+    for (int i = 0; i < kMergeCh; ++i) acc[i] += w * po[(size_t)i * kG];
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) tile[h][i] = acc[i] * inv;
+  for (int i = 0; i < kMergeCh; ++i) tile[h][i] = acc[i] * inv;
   if (blockIdx.x == 0)
     lse[(size_t)b * kG + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
   __syncthreads();
-  // write rows out[b][h][c0 .. c0+31]: 8 threads per head row, 4 floats each
-  for (int e = h; e < kG * 8; e += 128) {
-    const int hh = e >> 3, q4 = (e & 7) * 4;
+  // write rows out[b][h][c0 .. c0+7]: 2 threads per head row, 4 floats each
+  for (int e = h; e < kG * (kMergeCh / 4); e += 128) {
+    const int hh = e / (kMergeCh / 4), q4 = (e % (kMergeCh / 4)) * 4;
     *reinterpret_cast<float4*>(out + ((size_t)b * kG + hh) * kDv + c0 + q4) =
         make_float4(tile[hh][q4], tile[hh][q4 + 1], tile[hh][q4 + 2], tile[hh][q4 + 3]);
   }
@@ -757,7 +763,7 @@ cudaError_t launch_attend_mla(const sa_geom& g, const void* q, const void* kv,
   int ns = a.n_split;
   void* margs[] = {&po, &pml, &out, &lse, &ns};
   return launch_pdl_mla(reinterpret_cast<const void*>(attend_mla_merge_kernel),
-                        dim3(mla::kDv / 32, g.B), dim3(128), 0, stream, margs);
+                        dim3(mla::kDv / kMergeCh, g.B), dim3(128), 0, stream, margs);
 }
 
 }  // namespace sa
