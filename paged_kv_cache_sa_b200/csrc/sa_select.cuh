@@ -87,14 +87,27 @@ __device__ float warp_refresh_and_score(const uint4* __restrict__ k_cache,
   for (int g = 0; g < 8; ++g)
     qv[g] = (g < G && lane < CPR) ? *reinterpret_cast<const uint4*>(qh + (size_t)g * D + c * 8)
                                   : make_uint4(0, 0, 0, 0);
-#pragma unroll 4
-  for (int t = lane / CPR; t < valid; t += RPI) {
-    const uint4 v = __ldcg(blk + (size_t)t * CPR + c);
-    const uint32_t k0 = bf2_key(v.x), k1 = bf2_key(v.y), k2 = bf2_key(v.z), k3 = bf2_key(v.w);
-    mn.x = __vmins2(mn.x, k0); mn.y = __vmins2(mn.y, k1);
-    mn.z = __vmins2(mn.z, k2); mn.w = __vmins2(mn.w, k3);
-    mx.x = __vmaxs2(mx.x, k0); mx.y = __vmaxs2(mx.y, k1);
-    mx.z = __vmaxs2(mx.z, k2); mx.w = __vmaxs2(mx.w, k3);
+  // up to 16 rows per lane in flight at once (a whole page of 32 rows at Dk = 128): the
+  // refresh sits on its warp's critical path, so one memory round trip, not several
+  constexpr int kBatch = 16;
+  for (int t0 = lane / CPR; t0 < valid; t0 += kBatch * RPI) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int t = t0 + i * RPI;
+      if (t < valid) v[i] = __ldcg(blk + (size_t)t * CPR + c);
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      if (t0 + i * RPI < valid) {
+        const uint32_t k0 = bf2_key(v[i].x), k1 = bf2_key(v[i].y);
+        const uint32_t k2 = bf2_key(v[i].z), k3 = bf2_key(v[i].w);
+        mn.x = __vmins2(mn.x, k0); mn.y = __vmins2(mn.y, k1);
+        mn.z = __vmins2(mn.z, k2); mn.w = __vmins2(mn.w, k3);
+        mx.x = __vmaxs2(mx.x, k0); mx.y = __vmaxs2(mx.y, k1);
+        mx.z = __vmaxs2(mx.z, k2); mx.w = __vmaxs2(mx.w, k3);
+      }
+    }
   }
 #pragma unroll
   for (int off = CPR; off < 32; off <<= 1) {
