@@ -520,13 +520,8 @@ static size_t score_table_bytes(const sa_geom& g) {
 static void score_shape(const sa_geom& g, ScoreArgs* a, bool f8 = false) {
   const int D = g.Dk;
   const int G = g.Hq / g.Hkv;
-  int hg = 1;
-  if (!f8) {
-    while (hg < kScoreConsumers && g.Hkv % (hg * 2) == 0) hg *= 2;
-  } else {
-    // power of two dividing Hkv, at most 2 KB of bf16-equivalent summaries per slot
-    while (hg * 2 * 4 * D <= 2048 && g.Hkv % (hg * 2) == 0) hg *= 2;
-  }
+  int hg = 1;  // up to 8 KV heads per page slot: one bulk copy of their records per page
+  while (hg < kScoreConsumers && g.Hkv % (hg * 2) == 0) hg *= 2;
   a->HG = hg;
   a->n_hg = g.Hkv / hg;
   a->WPS = kScoreConsumers / hg;
@@ -548,18 +543,18 @@ static void score_shape(const sa_geom& g, ScoreArgs* a, bool f8 = false) {
     }
     a->NST = best;
   } else {
-    // half the bytes per stage: twice the stages in flight.  8-byte code loads of four
-    // page rows per half-warp are conflict-free when slots sit 32 B apart mod 128.
+    // 8-byte code loads of four page rows per half-warp are conflict-free when slots sit
+    // 32 B apart mod 128; as many stages as fit (a multiple of WPS, at most 8)
     a->rec_bytes = 2 * D + 16;
-    a->NST = 8;
     a->slot_bytes = ((hg * a->rec_bytes + 127) & ~127) + 32;
+    const int stage = (kTilePages * a->slot_bytes + hg * G * D * 2 + 127) & ~127;
+    int nst = (int)(limit / stage);
+    if (nst > 8) nst = 8;
+    nst -= nst % a->WPS;
+    a->NST = nst;
   }
   a->q_off = kTilePages * a->slot_bytes;
   a->stage_bytes = (a->q_off + hg * G * D * 2 + 127) & ~127;
-  // fp8: back to four stages when eight do not fit (large query groups)
-  if (f8 && a->WPS <= 4 &&
-      (size_t)8 * a->stage_bytes + score_table_bytes(g) > (size_t)kScoreSmemLimit)
-    a->NST = 4;
 }
 
 static size_t score_smem(const sa_geom& g, const ScoreArgs& a) {
@@ -587,7 +582,7 @@ bool score_supported_fp8(const sa_geom& g) {
   if (!(g.Dk == 64 || g.Dk == 128)) return false;
   ScoreArgs a;
   score_shape(g, &a, true);
-  return score_smem(g, a) <= (size_t)kScoreSmemLimit;
+  return a.NST >= 2 && score_smem(g, a) <= (size_t)kScoreSmemLimit;
 }
 
 static ScoreArgs make_score_args(const sa_geom& g, const void* q, const void* summ,
