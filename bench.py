@@ -584,8 +584,8 @@ def run_native(args, rank, world, dist):
             extras.update(extra_decode(name, args, dev, hbm_peak))
     # GQA: score, select (+ tail refresh), attention, merge; latent: tail refresh, query
     # sign split, tensor-core score, select, tensor-core attention, merge
-    # select half of one layer-call (fp8: the newest pages' records in a kernel of their own)
-    launches_select = 4 if g.v_aliases_k else (3 if F8 else 2)
+    # select half of one layer-call (the newest pages' refresh runs inside the scorer)
+    launches_select = 4 if g.v_aliases_k else 2
     launches_attend = 2                           # attention + merge
     launches_per_step = n_sel_layers * launches_select + L_layers * launches_attend
     line = {

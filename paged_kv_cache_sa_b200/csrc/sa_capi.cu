@@ -445,14 +445,12 @@ SA_EXPORT int sa_sparse_decode_fp8(const sa_geom* g, const void* q, const void* 
   int32_t* phys = reinterpret_cast<int32_t*>(w + plan.off_phys);
   float* scores = reinterpret_cast<float*>(w + plan.off_scores);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // newest pages' records first (their own kernel), then the fp8 scoring, the selection
-  // (nothing left to refresh) and the attention over bf16 K and V
-  if (n_tail_refresh > 0 &&
-      (st = cuda_status(launch_summaries_fp8(*g, k_cache, page_table, seq_lens, summ8,
-                                             n_tail_refresh, s))) != SA_OK)
-    return st;
+  // fp8 scoring (which first re-encodes the newest pages' records from K), the selection
+  // and the attention over bf16 K and V
   if ((st = cuda_status(launch_score(*g, q, summ8, page_table, seq_lens, scores,
-                                     plan.n_score_cta, status, s, true))) != SA_OK)
+                                     plan.n_score_cta, status, s, true,
+                                     n_tail_refresh > 0 ? k_cache : nullptr,
+                                     n_tail_refresh))) != SA_OK)
     return st;
   if ((st = cuda_status(launch_select(*g, page_table, seq_lens, scores, plan.K, sink / g->P,
                                       window / g->P, sel, cnt, phys, status, s))) != SA_OK)

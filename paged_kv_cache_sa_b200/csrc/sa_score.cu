@@ -32,9 +32,10 @@
 // (page, KV head): 2 * Dk + 16.
 //
 // Decode-time refresh: when asked, the consumer warps first recompute the summaries of
-// each sequence's newest pages from K (the pages that received appended tokens) and
-// score them, while the first copies are in flight; the stream skips those pages, so it
-// may read either version of their summaries.
+// each sequence's newest pages from K (the pages that received appended tokens; bf16
+// rows, or fp8 records encoded exactly as the summaries kernel encodes them) and score
+// them, while the first copies are in flight; the stream skips those pages, so it may
+// read either version of their summaries.
 //
 // Selection (select_kernel, one CTA per (sequence, KV head), launched programmatically
 // dependent on the scoring grid, which exits before it starts).  It turns the scores
@@ -51,6 +52,7 @@
 #include <cuda_fp8.h>
 
 #include "sa_common.cuh"
+#include "sa_fp8.cuh"
 #include "sa_internal.h"
 #include "sa_select.cuh"
 
@@ -71,8 +73,8 @@ struct ScoreArgs {
   const int32_t* seq_lens;
   float* scores;  // [B][Hkv][max_pages]
   int32_t* status;
-  const uint4* k_cache;  // bf16 summaries: refresh the newest n_tail pages from K first
-  uint4* summ_w;         // the summaries, written by that refresh
+  const uint4* k_cache;  // non-null: refresh the newest n_tail pages' summaries from K first
+  uint4* summ_w;         // the summaries (bf16 rows or fp8 records), written by that refresh
   int n_tail;
   int B, Hq, Hkv, G, P, max_pages, n_pool;
   int HG, n_hg, WPS, NST;              // heads per tile, head groups, warp groups, stages
@@ -104,6 +106,44 @@ __device__ __forceinline__ int find_seq(const int* pre, int n, int u) {
       hi = mid - 1;
   }
   return lo;
+}
+
+// fp8 form of the decode-time refresh (one warp): the page's min/max rows from K, encoded
+// into the record exactly as the summaries kernel encodes them and stored, and in every
+// lane the page's score over the decoded record (max over the G heads, then the
+// record's 2^e, as the stream applies it).
+template <int D>
+__device__ float warp_refresh_and_score_fp8(const uint4* __restrict__ k_cache,
+                                            uint8_t* __restrict__ summ8, const uint16_t* qh,
+                                            int G, int phys, int h, int Hkv, int P, int valid,
+                                            int lane) {
+  constexpr int CPR = D / 8;
+  uint4 qv[8];
+  warp_load_q<D>(qh, G, lane, qv);
+  uint4 kmin, kmax;
+  warp_page_minmax<D>(k_cache, phys, h, Hkv, P, valid, lane, kmin, kmax);
+  uint32_t am = max_mag2(max_mag2(max_mag2(max_mag2(0u, kmin.x), kmin.y), kmin.z), kmin.w);
+  am = max_mag2(max_mag2(max_mag2(max_mag2(am, kmax.x), kmax.y), kmax.z), kmax.w);
+  am = __reduce_max_sync(0xffffffffu, am);
+  const int e = fp8_record_exp(am);
+  const uint2 cmin = make_uint2(e4m3_pack(kmin.x, kmin.y, e, false),
+                                e4m3_pack(kmin.z, kmin.w, e, false));
+  const uint2 cmax = make_uint2(e4m3_pack(kmax.x, kmax.y, e, true),
+                                e4m3_pack(kmax.z, kmax.w, e, true));
+  uint8_t* rec = summ8 + ((size_t)phys * Hkv + h) * (2 * D + 16);
+  const int c = lane % CPR;
+  if (lane < CPR) {
+    *reinterpret_cast<uint2*>(rec + c * 8) = cmin;
+    *reinterpret_cast<uint2*>(rec + D + c * 8) = cmax;
+  }
+  if (lane == 0)
+    *reinterpret_cast<uint4*>(rec + 2 * D) = make_uint4((uint32_t)e & 0xFFu, 0u, 0u, 0u);
+  uint32_t lo[4], hi[4];
+  e4m3x4_to_bf16(cmin.x, lo[0], lo[1]);
+  e4m3x4_to_bf16(cmin.y, lo[2], lo[3]);
+  e4m3x4_to_bf16(cmax.x, hi[0], hi[1]);
+  e4m3x4_to_bf16(cmax.y, hi[2], hi[3]);
+  return ldexpf(warp_bound_score<D>(qv, G, lane, lo, hi), e);
 }
 
 // Tiles per sequence (n_hg * ceil(pages / 16)) prefix-summed over the batch by one warp;
@@ -257,7 +297,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
     //    received appended tokens), spread over the grid's consumer warps while the first
     //    copies are in flight.  Their scores replace the streamed ones (the stream skips
     //    those pages), so the stream may read either version of the summaries.
-    if constexpr (!F8) {
+    {
       const int n_items = a.B * a.Hkv * a.n_tail;
       for (int i = c + n_cta * warp; i < n_items; i += n_cta * kScoreConsumers) {
         const int pr = i / a.n_tail;
@@ -267,10 +307,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const Sc
         if (lp < 0) continue;
         const int ph = a.page_table[(size_t)b * a.max_pages + lp];
         float sc = 0.f;
-        if (ph >= 0 && ph < a.n_pool)
-          sc = warp_refresh_and_score<D>(a.k_cache, a.summ_w,
-                                         a.q + ((size_t)b * a.Hq + h * a.G) * D, a.G, ph, h,
-                                         a.Hkv, a.P, min(a.P, L - lp * a.P), lane);
+        if (ph >= 0 && ph < a.n_pool) {
+          const uint16_t* qh = a.q + ((size_t)b * a.Hq + h * a.G) * D;
+          const int valid = min(a.P, L - lp * a.P);
+          if constexpr (F8)
+            sc = warp_refresh_and_score_fp8<D>(a.k_cache, reinterpret_cast<uint8_t*>(a.summ_w),
+                                               qh, a.G, ph, h, a.Hkv, a.P, valid, lane);
+          else
+            sc = warp_refresh_and_score<D>(a.k_cache, a.summ_w, qh, a.G, ph, h, a.Hkv, a.P,
+                                           valid, lane);
+        }
         if (lane == 0) a.scores[(size_t)pr * a.max_pages + lp] = sc;
       }
     }
@@ -614,7 +660,7 @@ cudaError_t launch_score(const sa_geom& g, const void* q, const void* summ,
                          int n_cta, int32_t* status, cudaStream_t stream, bool fp8,
                          const void* k_cache, int n_tail) {
   ScoreArgs a = make_score_args(g, q, summ, page_table, seq_lens, scores, status, fp8);
-  if (!fp8 && k_cache && n_tail > 0) {
+  if (k_cache && n_tail > 0) {
     a.k_cache = static_cast<const uint4*>(k_cache);
     a.summ_w = static_cast<uint4*>(const_cast<void*>(summ));
     a.n_tail = n_tail < kMaxTail ? n_tail : kMaxTail;

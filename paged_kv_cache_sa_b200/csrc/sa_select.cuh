@@ -69,24 +69,33 @@ __device__ __forceinline__ int sel_block_excl_scan(int v, int* warp_tot, int* to
   return res;
 }
 
-// Recompute the summary of one (physical page, KV head) from K (one warp), store it,
-// and return in every lane its score for the G query heads at qh (max over heads).
+// Pieces of the decode-time refresh of one (physical page, KV head), one warp: lane l
+// works on 16-byte chunk l % (D / 8) of the rows.
+
+// The G <= 8 query rows at qh (chunk of this lane; zero past G).  Loaded before K so
+// that their loads are in flight together.
 template <int D>
-__device__ float warp_refresh_and_score(const uint4* __restrict__ k_cache,
-                                        uint4* __restrict__ summ, const uint16_t* qh, int G,
-                                        int phys, int h, int Hkv, int P, int valid, int lane) {
+__device__ __forceinline__ void warp_load_q(const uint16_t* qh, int G, int lane, uint4 (&qv)[8]) {
+  constexpr int CPR = D / 8;
+#pragma unroll
+  for (int g = 0; g < 8; ++g)
+    qv[g] = (g < G && lane < CPR)
+                ? *reinterpret_cast<const uint4*>(qh + (size_t)g * D + (lane % CPR) * 8)
+                : make_uint4(0, 0, 0, 0);
+}
+
+// Channel-wise min and max (bf16 patterns) of the page's `valid` rows of K; every lane
+// ends with those of its chunk.
+template <int D>
+__device__ __forceinline__ void warp_page_minmax(const uint4* __restrict__ k_cache, int phys,
+                                                 int h, int Hkv, int P, int valid, int lane,
+                                                 uint4& kmin, uint4& kmax) {
   constexpr int CPR = D / 8;     // 8 or 16 chunks per row
   constexpr int RPI = 32 / CPR;  // rows per warp iteration
   const int c = lane % CPR;
   const uint4* blk = k_cache + ((size_t)phys * Hkv + h) * P * CPR;
   uint4 mn = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
   uint4 mx = make_uint4(0x80008000u, 0x80008000u, 0x80008000u, 0x80008000u);
-  // query rows first: independent of K, so their loads are in flight with K's
-  uint4 qv[8];
-#pragma unroll
-  for (int g = 0; g < 8; ++g)
-    qv[g] = (g < G && lane < CPR) ? *reinterpret_cast<const uint4*>(qh + (size_t)g * D + c * 8)
-                                  : make_uint4(0, 0, 0, 0);
   // up to 16 rows per lane in flight at once (a whole page of 32 rows at Dk = 128): the
   // refresh sits on its warp's critical path, so one memory round trip, not several
   constexpr int kBatch = 16;
@@ -120,15 +129,17 @@ __device__ float warp_refresh_and_score(const uint4* __restrict__ k_cache,
     mx.z = __vmaxs2(mx.z, __shfl_xor_sync(0xffffffffu, mx.z, off));
     mx.w = __vmaxs2(mx.w, __shfl_xor_sync(0xffffffffu, mx.w, off));
   }
-  const uint4 kmin = make_uint4(bf2_key(mn.x), bf2_key(mn.y), bf2_key(mn.z), bf2_key(mn.w));
-  const uint4 kmax = make_uint4(bf2_key(mx.x), bf2_key(mx.y), bf2_key(mx.z), bf2_key(mx.w));
-  uint4* out = summ + ((size_t)phys * Hkv + h) * 2 * CPR;
-  if (lane < CPR) {
-    __stcg(out + c, kmin);
-    __stcg(out + CPR + c, kmax);
-  }
-  const uint32_t lo[4] = {kmin.x, kmin.y, kmin.z, kmin.w};
-  const uint32_t hi[4] = {kmax.x, kmax.y, kmax.z, kmax.w};
+  kmin = make_uint4(bf2_key(mn.x), bf2_key(mn.y), bf2_key(mn.z), bf2_key(mn.w));
+  kmax = make_uint4(bf2_key(mx.x), bf2_key(mx.y), bf2_key(mx.z), bf2_key(mx.w));
+}
+
+// max over the G query heads of sum_c max(q_gc * hi_c, q_gc * lo_c), lo/hi the bf16
+// pairs of this lane's 8 channels (lanes past the row add nothing); in every lane.
+template <int D>
+__device__ __forceinline__ float warp_bound_score(const uint4 (&qv)[8], int G, int lane,
+                                                  const uint32_t (&lo)[4],
+                                                  const uint32_t (&hi)[4]) {
+  constexpr int CPR = D / 8;
   float best = -INFINITY;
 #pragma unroll
   for (int g = 0; g < 8; ++g) {
@@ -152,6 +163,28 @@ __device__ float warp_refresh_and_score(const uint4* __restrict__ k_cache,
     best = fmaxf(best, part);
   }
   return best;
+}
+
+// Recompute the bf16 summary of one (physical page, KV head) from K (one warp), store
+// it, and return in every lane its score for the G query heads at qh (max over heads).
+template <int D>
+__device__ float warp_refresh_and_score(const uint4* __restrict__ k_cache,
+                                        uint4* __restrict__ summ, const uint16_t* qh, int G,
+                                        int phys, int h, int Hkv, int P, int valid, int lane) {
+  constexpr int CPR = D / 8;
+  uint4 qv[8];
+  warp_load_q<D>(qh, G, lane, qv);
+  uint4 kmin, kmax;
+  warp_page_minmax<D>(k_cache, phys, h, Hkv, P, valid, lane, kmin, kmax);
+  uint4* out = summ + ((size_t)phys * Hkv + h) * 2 * CPR;
+  const int c = lane % CPR;
+  if (lane < CPR) {
+    __stcg(out + c, kmin);
+    __stcg(out + CPR + c, kmax);
+  }
+  const uint32_t lo[4] = {kmin.x, kmin.y, kmin.z, kmin.w};
+  const uint32_t hi[4] = {kmax.x, kmax.y, kmax.z, kmax.w};
+  return warp_bound_score<D>(qv, G, lane, lo, hi);
 }
 
 // Threshold of the top-k_rem0 candidates among keys[0, nb) (forced pages, p < s_pages or
