@@ -204,8 +204,10 @@ int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache, const
  * bf16 exactly; products exact; fp32 accumulation), -inf beyond each sequence.
  * sa_sparse_decode_fp8: sa_sparse_decode with the selection scored over fp8 records;
  * attention still reads the bf16 K and V.  n_tail_refresh (0..16) re-encodes the
- * newest pages' records from k_cache first (a kernel of its own).  Argument rules and
- * workspace as for sa_sparse_decode (summ8 16-byte aligned).
+ * newest pages' records from k_cache first, exactly as sa_update_summaries_fp8 would
+ * (inside the scoring kernel; a refreshed page must not be shared with another sequence
+ * of the call).  Argument rules and workspace as for sa_sparse_decode (summ8 16-byte
+ * aligned).
  * ------------------------------------------------------------------------------ */
 size_t sa_summary_fp8_record_bytes(const sa_geom* g);
 int sa_page_summaries_fp8(const sa_geom* g, const void* k_cache, const int32_t* page_table,
