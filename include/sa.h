@@ -186,6 +186,26 @@ int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_cache, const
                      size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * sa_sparse_decode_fused: the same outputs as sa_sparse_decode (grouped-query geometry,
+ * V not aliasing K) from one persistent launch instead of four kernels: page scoring
+ * with the n_tail_refresh refresh, the selection, the gathered attention and the merge
+ * run as phases of one grid of one CTA per SM, all resident (cooperative launch), handed
+ * over by grid barriers on a counter in the workspace header (zeroed on `stream` before
+ * the launch; a barrier that waits longer than 2 s sets SA_ERR_TIMEOUT).  The selection
+ * is bit-identical to sa_sparse_decode's; the attention is the same computation with the
+ * same work split.  SA_ERR_UNSUPPORTED where one CTA per SM cannot cover the geometry
+ * or the phases' shared memory does not fit.  Arguments and workspace as for
+ * sa_sparse_decode.  [VX section 1; SSA section; FlashAttention paragraph: the method
+ * of (4), in one launch.]
+ * ------------------------------------------------------------------------------ */
+int sa_sparse_decode_fused(const sa_geom* g, const void* q, const void* k_cache,
+                           const void* v_cache, void* summ, const int32_t* page_table,
+                           const int32_t* seq_lens, int budget, int sink, int window,
+                           int n_tail_refresh, float scale, float* out, float* lse,
+                           int32_t* sel_out, int32_t* sel_count_out, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* ---------------------------------------------------------------------------------
  * fp8 summaries rounded outward (grouped-query geometry only; others return
  * SA_ERR_UNSUPPORTED)  [SE hook-point paragraph: quantised KV (KIVI) listed next to
  * Quest; the pages give no format].  Per (physical page, KV head) a record of

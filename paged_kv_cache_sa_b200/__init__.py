@@ -44,7 +44,7 @@ EXPORTS = ["sa_status_string", "sa_version", "sa_decode_workspace_size", "sa_pru
            "sa_page_scores", "sa_select_pages", "sa_sparse_decode", "sa_attend_selected",
            "sa_prune_compact", "sa_sparse_decode_noalloc", "sa_summary_fp8_record_bytes",
            "sa_page_summaries_fp8", "sa_update_summaries_fp8", "sa_page_scores_fp8",
-           "sa_sparse_decode_fp8"]
+           "sa_sparse_decode_fp8", "sa_sparse_decode_fused"]
 
 
 class SaError(RuntimeError):
@@ -100,6 +100,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                              vp], i32),
         "sa_sparse_decode": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, vp,
                               vp, vp, vp, vp, sz, vp], i32),
+        "sa_sparse_decode_fused": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                    ctypes.c_float, vp, vp, vp, vp, vp, sz, vp], i32),
         "sa_sparse_decode_noalloc": ([G, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                       ctypes.c_float, vp, vp, vp, vp, vp, vp], i32),
         "sa_summary_fp8_record_bytes": ([G], sz),
@@ -242,6 +244,25 @@ def sparse_decode(geom: Geometry, q, k_cache, v_cache, summ, page_table, seq_len
                                 int(window), int(n_tail_refresh), float(scale), _ptr(out),
                                 _ptr(lse), _ptr(sel_out), _ptr(sel_count_out), _ptr(ws.buf),
                                 ws.nbytes, _stream(stream)), "sa_sparse_decode")
+    return out, lse
+
+
+def sparse_decode_fused(geom: Geometry, q, k_cache, v_cache, summ, page_table, seq_lens, budget,
+                        sink, window, scale, ws: Workspace, out=None, lse=None, sel_out=None,
+                        sel_count_out=None, n_tail_refresh: int = 0, stream=None):
+    """sparse_decode in one persistent launch (grouped-query geometry)."""
+    dev = q.device
+    if out is None:
+        out = torch.empty((geom.B, geom.Hq, geom.Dv), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((geom.B, geom.Hq), dtype=torch.float32, device=dev)
+    g = geom.c()
+    _check(lib.sa_sparse_decode_fused(ctypes.byref(g), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(summ), _ptr(page_table), _ptr(seq_lens), int(budget),
+                                      int(sink), int(window), int(n_tail_refresh),
+                                      float(scale), _ptr(out), _ptr(lse), _ptr(sel_out),
+                                      _ptr(sel_count_out), _ptr(ws.buf), ws.nbytes,
+                                      _stream(stream)), "sa_sparse_decode_fused")
     return out, lse
 
 

@@ -371,6 +371,58 @@ SA_EXPORT int sa_sparse_decode(const sa_geom* g, const void* q, const void* k_ca
   return run_attend(*g, plan, w, q, k_cache, vc, page_table, seq_lens, sel, cnt,
                     reinterpret_cast<int32_t*>(w + plan.off_phys), plan.K, scale, out, lse, s);
 }
+SA_EXPORT int sa_sparse_decode_fused(const sa_geom* g, const void* q, const void* k_cache,
+                                     const void* v_cache, void* summ, const int32_t* page_table,
+                                     const int32_t* seq_lens, int budget, int sink, int window,
+                                     int n_tail_refresh, float scale, float* out, float* lse,
+                                     int32_t* sel_out, int32_t* sel_count_out, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  int st = check_geom(g);
+  if (st != SA_OK) return st;
+  if ((st = check_budget(*g, budget, sink, window)) != SA_OK) return st;
+  if (!q || !k_cache || !v_cache || !summ || !page_table || !seq_lens || !out || !lse)
+    return SA_ERR_INVALID_ARG;
+  if (n_tail_refresh < 0 || n_tail_refresh > 16) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(summ))
+    return SA_ERR_INVALID_ARG;
+  if ((size_t)g->max_pages * 4 > 200 * 1024) return SA_ERR_UNSUPPORTED;
+  if (!is_gqa(*g) || g->v_aliases_k) return SA_ERR_UNSUPPORTED;
+  DecodePlan plan;
+  make_decode_plan(*g, budget, &plan);
+  if (!ws || ws_bytes < plan.total || !aligned16(ws)) return SA_ERR_WORKSPACE;
+  if (!fused_supported(*g, plan.K, plan.n_sm)) return SA_ERR_UNSUPPORTED;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
+  FusedCall f;
+  f.q = q;
+  f.k_cache = k_cache;
+  f.v_cache = v_cache;
+  f.summ = summ;
+  f.page_table = page_table;
+  f.seq_lens = seq_lens;
+  f.K = plan.K;
+  f.s_pages = sink / g->P;
+  f.w_pages = window / g->P;
+  f.n_tail = n_tail_refresh;
+  f.scale = scale;
+  f.scores = reinterpret_cast<float*>(w + plan.off_scores);
+  f.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + plan.off_sel);
+  f.sel_count = sel_count_out ? sel_count_out : reinterpret_cast<int32_t*>(w + plan.off_cnt);
+  f.sel_phys = reinterpret_cast<int32_t*>(w + plan.off_phys);
+  f.part = reinterpret_cast<float*>(w + plan.off_part);
+  f.pre = reinterpret_cast<int32_t*>(w + plan.off_pre);
+  f.out = out;
+  f.lse = lse;
+  f.status = &hdr->status_bits;
+  f.counter = &hdr->pad[0];
+  f.n_cta = plan.n_sm;
+  f.n_sm = plan.n_sm;
+  const cudaError_t e = launch_fused(*g, f, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorInvalidConfiguration)
+    return SA_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
 // ---- fp8 summaries rounded outward (grouped-query geometry) ---------------------------
 
 SA_EXPORT size_t sa_summary_fp8_record_bytes(const sa_geom* g) {

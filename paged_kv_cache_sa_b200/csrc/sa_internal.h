@@ -85,6 +85,32 @@ struct AttendCall {
   int counts_from_lens;  // the selection came from this library for these seq_lens
 };
 
+// the whole grouped-query decode step in one persistent launch
+struct FusedCall {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  void* summ;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  int K, s_pages, w_pages, n_tail;
+  float scale;
+  float* scores;
+  int32_t* sel;
+  int32_t* sel_count;
+  int32_t* sel_phys;
+  float* part;
+  int32_t* pre;
+  float* out;
+  float* lse;
+  int32_t* status;
+  int32_t* counter;  // grid-barrier counter (zeroed on the stream before the launch)
+  int n_cta, n_sm;
+};
+
+bool fused_supported(const sa_geom& g, int K, int n_sm);
+cudaError_t launch_fused(const sa_geom& g, const FusedCall& f, cudaStream_t stream);
+
 int attend_ctas(const sa_geom& g, int K, int sms);
 size_t attend_partial_floats(const sa_geom& g, int n_cta);
 bool attend_supported(const sa_geom& g);

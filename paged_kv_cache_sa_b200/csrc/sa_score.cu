@@ -47,389 +47,19 @@
 // asc) and the winners marked; all-equal boundary keys take the lowest pages.  The
 // ascending list of forced and taken pages (and their physical ids) is written with
 // per-warp ballots and one block barrier.  Deterministic.
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-#include <cuda_fp8.h>
-
-#include "sa_common.cuh"
-#include "sa_fp8.cuh"
-#include "sa_internal.h"
-#include "sa_select.cuh"
+#include "sa_attend.cuh"
+#include "sa_score.cuh"
 
 namespace sa {
 
-constexpr int kTilePages = 16;  // pages per tile: the M side of one MMA
-constexpr int kScoreConsumers = 8;
-constexpr int kScoreThreads = (kScoreConsumers + 1) * 32;
-constexpr int kMaxTilesPerCta = 64;
-constexpr int kSlotPad = 64;  // odd multiple of 64 B between page slots: no bank conflicts
-constexpr int kSelectThreads = 512;
-constexpr int kScoreSmemLimit = 227 * 1024;
-
-struct ScoreArgs {
-  const uint16_t* q;
-  const uint8_t* summ;
-  const int32_t* page_table;
-  const int32_t* seq_lens;
-  float* scores;  // [B][Hkv][max_pages]
-  int32_t* status;
-  const uint4* k_cache;  // non-null: refresh the newest n_tail pages' summaries from K first
-  uint4* summ_w;         // the summaries (bf16 rows or fp8 records), written by that refresh
-  int n_tail;
-  int B, Hq, Hkv, G, P, max_pages, n_pool;
-  int HG, n_hg, WPS, NST;              // heads per tile, head groups, warp groups, stages
-  int slot_bytes, q_off, stage_bytes;  // stage: [16][slot_bytes] page slots | q rows
-  int rec_bytes;                       // summary bytes per (page, KV head)
-};
-
-// Four E4M3 codes (bytes of w, lowest first) as two bf16x2 words, exactly: the
-// hardware e4m3x2 -> f16x2 conversion, then f16 -> f32 -> bf16 (no rounding anywhere:
-// every E4M3 value has at most 4 significant bits within the exponent range of both).
-__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const __half2 a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
-  const __half2 b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-  const float2 fa = __half22float2(a), fb = __half22float2(b);
-  const __nv_bfloat162 ba = __floats2bfloat162_rn(fa.x, fa.y);
-  const __nv_bfloat162 bb = __floats2bfloat162_rn(fb.x, fb.y);
-  lo = *reinterpret_cast<const uint32_t*>(&ba);
-  hi = *reinterpret_cast<const uint32_t*>(&bb);
-}
-
-// the sequence owning flattened tile u: largest b with pre[b] <= u
-__device__ __forceinline__ int find_seq(const int* pre, int n, int u) {
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (pre[mid] <= u)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  return lo;
-}
-
-// fp8 form of the decode-time refresh (one warp): the page's min/max rows from K, encoded
-// into the record exactly as the summaries kernel encodes them and stored, and in every
-// lane the page's score over the decoded record (max over the G heads, then the
-// record's 2^e, as the stream applies it).
-template <int D>
-__device__ float warp_refresh_and_score_fp8(const uint4* __restrict__ k_cache,
-                                            uint8_t* __restrict__ summ8, const uint16_t* qh,
-                                            int G, int phys, int h, int Hkv, int P, int valid,
-                                            int lane) {
-  constexpr int CPR = D / 8;
-  uint4 qv[8];
-  warp_load_q<D>(qh, G, lane, qv);
-  uint4 kmin, kmax;
-  warp_page_minmax<D>(k_cache, phys, h, Hkv, P, valid, lane, kmin, kmax);
-  uint32_t am = max_mag2(max_mag2(max_mag2(max_mag2(0u, kmin.x), kmin.y), kmin.z), kmin.w);
-  am = max_mag2(max_mag2(max_mag2(max_mag2(am, kmax.x), kmax.y), kmax.z), kmax.w);
-  am = __reduce_max_sync(0xffffffffu, am);
-  const int e = fp8_record_exp(am);
-  const uint2 cmin = make_uint2(e4m3_pack(kmin.x, kmin.y, e, false),
-                                e4m3_pack(kmin.z, kmin.w, e, false));
-  const uint2 cmax = make_uint2(e4m3_pack(kmax.x, kmax.y, e, true),
-                                e4m3_pack(kmax.z, kmax.w, e, true));
-  uint8_t* rec = summ8 + ((size_t)phys * Hkv + h) * (2 * D + 16);
-  const int c = lane % CPR;
-  if (lane < CPR) {
-    *reinterpret_cast<uint2*>(rec + c * 8) = cmin;
-    *reinterpret_cast<uint2*>(rec + D + c * 8) = cmax;
-  }
-  if (lane == 0)
-    *reinterpret_cast<uint4*>(rec + 2 * D) = make_uint4((uint32_t)e & 0xFFu, 0u, 0u, 0u);
-  uint32_t lo[4], hi[4];
-  e4m3x4_to_bf16(cmin.x, lo[0], lo[1]);
-  e4m3x4_to_bf16(cmin.y, lo[2], lo[3]);
-  e4m3x4_to_bf16(cmax.x, hi[0], hi[1]);
-  e4m3x4_to_bf16(cmax.y, hi[2], hi[3]);
-  return ldexpf(warp_bound_score<D>(qv, G, lane, lo, hi), e);
-}
-
-// Tiles per sequence (n_hg * ceil(pages / 16)) prefix-summed over the batch by one warp;
-// returns the total.  With pre/nbs non-null the prefix and page counts are stored.
-__device__ __forceinline__ int tile_prefix(const ScoreArgs& a, int lane, int* pre, int* nbs) {
-  int carry = 0;
-  for (int b0 = 0; b0 < a.B; b0 += 32) {
-    const int b = b0 + lane;
-    int n = 0;
-    if (b < a.B) {
-      const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
-      const int nb = (L + a.P - 1) / a.P;
-      n = a.n_hg * ((nb + kTilePages - 1) / kTilePages);
-      if (nbs) nbs[b] = nb;
-    }
-    int incl = n;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    if (pre && b < a.B) pre[b] = carry + incl - n;
-    carry += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  if (pre && lane == 0) pre[a.B] = carry;
-  return carry;
-}
-
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
-
 template <int D, bool F8 = false>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_stream_kernel(const ScoreArgs a) {
-  constexpr int J = D / 16;  // 16-byte chunks per lane of the 2*D-long contraction row
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* stages = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  int* pre = reinterpret_cast<int*>(stages + (size_t)a.NST * a.stage_bytes);  // [B + 1]
-  int* nbs = pre + a.B + 1;                        // [B] pages per sequence
-  int* ptab = nbs + a.B;                           // [kMaxTilesPerCta * 16]
-  int* t_b = ptab + kMaxTilesPerCta * kTilePages;  // per tile of the slice
-  int* t_hg = t_b + kMaxTilesPerCta;
-  int* t_p0 = t_hg + kMaxTilesPerCta;
-  int* t_np = t_p0 + kMaxTilesPerCta;  // pages in the tile
-  int* t_vm = t_np + kMaxTilesPerCta;  // mask of pages with a valid slot
-  __shared__ __align__(8) uint64_t full_bar[8];
-  __shared__ __align__(8) uint64_t empty_bar[8];
-  __shared__ int abort_flag;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = blockIdx.x, n_cta = gridDim.x;
-
-  if (tid == 0) {
-    for (int s = 0; s < a.NST; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], a.HG);
-    }
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  // everything read below may come from the previous kernel of the stream: one thread
-  // waits for it (which makes its memory visible to this grid), the rest block on the
-  // CTA barrier.  No early launch of the next grid: the selection grid would start while
-  // most SMs still stream, and its CTAs would pile onto the first SMs to free up (several
-  // per SM, contending); launched as this grid exits, they spread over idle SMs.
-  if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
-  __syncthreads();
-
-  // The slice of the flattened tile list this CTA streams: every warp derives it from
-  // the sequence lengths itself, so no CTA-wide barrier stands before the first copy.
-  // Per-tile tables are written by the producer before it arrives on the tile's stage
-  // barrier (release), and read by the consumers after waiting on it (acquire).
-  const bool is_prod = warp == kScoreConsumers;
-  const int total = tile_prefix(a, lane, is_prod ? pre : nullptr, is_prod ? nbs : nullptr);
-  const int W = max(1, (total + n_cta - 1) / n_cta);
-  const int T0 = min(total, c * W);
-  const int nt = min(total, T0 + W) - T0;  // <= kMaxTilesPerCta (the host sizes the grid)
-
-  if (is_prod) {
-    // ===================== producer warp =====================
-    __syncwarp();
-    // 1. per tile of the slice (one lane each): sequence, head group, first page, page
-    //    count; its page-table entries gathered by asynchronous 4-byte copies, all in
-    //    flight together
-    for (int i = lane; i < nt; i += 32) {
-      const int u = T0 + i;
-      const int b = find_seq(pre, a.B, u);
-      const int ntb = (pre[b + 1] - pre[b]) / a.n_hg;  // tiles per head group
-      const int rem = u - pre[b];
-      const int p0 = (rem % ntb) * kTilePages;
-      const int np = min(kTilePages, nbs[b] - p0);
-      t_b[i] = b;
-      t_hg[i] = rem / ntb;
-      t_p0[i] = p0;
-      t_np[i] = np;
-      const int32_t* src = a.page_table + (size_t)b * a.max_pages + p0;
-      for (int pg = 0; pg < np; ++pg) cp_async4(ptab + i * kTilePages + pg, src + pg);
-    }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
-    __syncwarp();
-
-    // 2. bulk-copy issue: lanes 0-15 check and copy one page each, lane 16 the queries
-    const uint32_t slot_data = (uint32_t)a.HG * a.rec_bytes;  // one page's records of the group
-    const uint32_t q_bytes = (uint32_t)a.HG * a.G * D * 2;
-    uint64_t t_idle = 0;
-    const uint64_t ef = l2_evict_first();
-    for (int k = 0; k < nt;) {
-      const int s = k % a.NST;
-      bool ready = k < a.NST;
-      if (!ready && lane == 0) ready = mbar_test(&empty_bar[s], ((k / a.NST) - 1) & 1);
-      ready = __shfl_sync(0xffffffffu, ready, 0);
-      if (!ready) {
-        const uint64_t now = global_ns();
-        if (t_idle == 0) t_idle = now;
-        const int to = (now - t_idle > kWaitLimitNs) || *(volatile int*)&abort_flag;
-        if (__shfl_sync(0xffffffffu, to, 0)) {
-          if (lane == 0) {
-            report(a.status, SA_ERR_TIMEOUT);
-            atomicExch(&abort_flag, 1);
-          }
-          break;
-        }
-        continue;
-      }
-      t_idle = 0;
-      const int b = t_b[k], hg = t_hg[k], np = t_np[k];
-      const int ph = lane < np ? ptab[k * kTilePages + lane] : -1;
-      const bool ok = ph >= 0 && ph < a.n_pool;
-      if (lane < np && !ok) report(a.status, SA_ERR_DEVICE_CHECK);
-      const int vm = (int)(__ballot_sync(0xffffffffu, ok) & 0xFFFFu);
-      uint8_t* st = stages + (size_t)s * a.stage_bytes;
-      if (lane == 0) {
-        t_vm[k] = vm;
-        mbar_arrive_expect_tx(&full_bar[s], __popc(vm) * slot_data + q_bytes);
-      }
-      __syncwarp();
-      if (ok) {
-        bulk_load_hint(st + lane * a.slot_bytes,
-                       a.summ + ((size_t)ph * a.Hkv + hg * a.HG) * (size_t)a.rec_bytes,
-                       slot_data, &full_bar[s], ef);
-      } else if (lane == kTilePages) {
-        bulk_load(st + a.q_off, a.q + ((size_t)b * a.Hq + (size_t)hg * a.HG * a.G) * D, q_bytes,
-                  &full_bar[s]);
-      }
-      ++k;
-    }
-  } else {
-    // ===================== consumer warps =====================
-    // 0. decode-time refresh of the newest pages' summaries from K (the pages that
-    //    received appended tokens), spread over the grid's consumer warps while the first
-    //    copies are in flight.  Their scores replace the streamed ones (the stream skips
-    //    those pages), so the stream may read either version of the summaries.
-    {
-      const int n_items = a.B * a.Hkv * a.n_tail;
-      for (int i = c + n_cta * warp; i < n_items; i += n_cta * kScoreConsumers) {
-        const int pr = i / a.n_tail;
-        const int b = pr / a.Hkv, h = pr % a.Hkv;
-        const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
-        const int lp = (L + a.P - 1) / a.P - a.n_tail + i % a.n_tail;
-        if (lp < 0) continue;
-        const int ph = a.page_table[(size_t)b * a.max_pages + lp];
-        float sc = 0.f;
-        if (ph >= 0 && ph < a.n_pool) {
-          const uint16_t* qh = a.q + ((size_t)b * a.Hq + h * a.G) * D;
-          const int valid = min(a.P, L - lp * a.P);
-          if constexpr (F8)
-            sc = warp_refresh_and_score_fp8<D>(a.k_cache, reinterpret_cast<uint8_t*>(a.summ_w),
-                                               qh, a.G, ph, h, a.Hkv, a.P, valid, lane);
-          else
-            sc = warp_refresh_and_score<D>(a.k_cache, a.summ_w, qh, a.G, ph, h, a.Hkv, a.P,
-                                           valid, lane);
-        }
-        if (lane == 0) a.scores[(size_t)pr * a.max_pages + lp] = sc;
-      }
-    }
-    const int r = lane >> 2, t = lane & 3;
-    const int grp = warp / a.HG, hh = warp % a.HG;  // stage group, head within the group
-    const bool v0 = 2 * t < a.G, v1 = 2 * t + 1 < a.G;
-    for (int k = grp; k < nt; k += a.WPS) {
-      const int s = k % a.NST;
-      bool ok = !*(volatile int*)&abort_flag;
-      if (ok && !mbar_wait(&full_bar[s], (k / a.NST) & 1)) {
-        report(a.status, SA_ERR_TIMEOUT);
-        atomicExch(&abort_flag, 1);
-        ok = false;
-      }
-      if (ok) {
-        const int b = t_b[k], h = t_hg[k] * a.HG + hh, p0 = t_p0[k], np = t_np[k];
-        const int vm = t_vm[k];
-        const uint32_t st = smem_u32(stages + (size_t)s * a.stage_bytes);
-        // B: [min(q,0) | max(q,0)] of query head n = r of KV head h, chunk 4j + t
-        uint32_t bq[J][4];
-        const uint32_t qrow = st + a.q_off + (uint32_t)(hh * a.G + (r < a.G ? r : 0)) * D * 2;
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-          const int cc = 4 * j + t;  // chunk of the 2D-long contraction
-          const uint4 v = lds_v4(qrow + (cc % (D / 8)) * 16);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t neg = ((w[e] >> 15) & 0x00010001u) * 0xFFFFu;  // negative halves
-            bq[j][e] = r < a.G ? ((cc < D / 8) ? (w[e] & neg) : (w[e] & ~neg)) : 0u;
-          }
-        }
-        // A: rows r and r + 8 of the tile (pages p0 + r, p0 + r + 8)
-        const bool va = (vm >> r) & 1, vb = (vm >> (r + 8)) & 1;
-        const uint32_t rowa = st + r * a.slot_bytes + hh * a.rec_bytes;
-        const uint32_t rowb = rowa + 8 * a.slot_bytes;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-          uint4 ra, rb;
-          if constexpr (F8) {
-            // chunk 4j + t of the contraction = 8 codes (channels of the same q chunk)
-            const uint2 ca = va ? lds_v2(rowa + (4 * j + t) * 8) : make_uint2(0, 0);
-            const uint2 cb = vb ? lds_v2(rowb + (4 * j + t) * 8) : make_uint2(0, 0);
-            e4m3x4_to_bf16(ca.x, ra.x, ra.y);
-            e4m3x4_to_bf16(ca.y, ra.z, ra.w);
-            e4m3x4_to_bf16(cb.x, rb.x, rb.y);
-            e4m3x4_to_bf16(cb.y, rb.z, rb.w);
-          } else {
-            ra = va ? lds_v4(rowa + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
-            rb = vb ? lds_v4(rowb + (4 * j + t) * 16) : make_uint4(0, 0, 0, 0);
-          }
-          mma_bf16_16816(acc, ra.x, rb.x, ra.y, rb.y, bq[j][0], bq[j][1]);
-          mma_bf16_16816(acc, ra.z, rb.z, ra.w, rb.w, bq[j][2], bq[j][3]);
-        }
-        // acc: [page r][heads 2t, 2t+1], [page r+8][heads 2t, 2t+1]
-        float m0 = fmaxf(v0 ? acc[0] : -INFINITY, v1 ? acc[1] : -INFINITY);
-        float m1 = fmaxf(v0 ? acc[2] : -INFINITY, v1 ? acc[3] : -INFINITY);
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
-        if constexpr (F8) {
-          // the records' exponents (an invalid page scored 0 stays 0)
-          const uint8_t* sp = stages + (size_t)s * a.stage_bytes + hh * a.rec_bytes + 2 * D;
-          m0 = ldexpf(m0, (int)(int8_t)sp[r * a.slot_bytes]);
-          m1 = ldexpf(m1, (int)(int8_t)sp[(r + 8) * a.slot_bytes]);
-        }
-        if (t == 0) {
-          // pages refreshed above keep the score computed from their fresh summary
-          const int lim = a.n_tail > 0 ? min(np, nbs[b] - a.n_tail - p0) : np;
-          float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages + p0;
-          if (r < lim) srow[r] = m0;
-          if (r + 8 < lim) srow[r + 8] = m1;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
-    }
-  }
-  if (warp == kScoreConsumers) {
-    // scores past each sequence's last page are -inf (pairs spread over the CTAs)
-    for (int pr = c; pr < a.B * a.Hkv; pr += n_cta) {
-      const int b = pr / a.Hkv;
-      const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
-      float* srow = a.scores + (size_t)pr * a.max_pages;
-      for (int p = (L + a.P - 1) / a.P + lane; p < a.max_pages; p += 32) srow[p] = -INFINITY;
-    }
-  }
-  __syncthreads();
-  if (abort_flag && warp == kScoreConsumers && lane == 0) {
-    // a wait expired: give copies still in flight a bounded time (10 ms) to land
-    const uint64_t t0 = global_ns();
-    while (global_ns() - t0 < 10000000ull) {
-    }
-  }
+  score_stream_body<D, F8>(a, smem_raw);
 }
-
-struct SelectArgs {
-  const int32_t* page_table;
-  const int32_t* seq_lens;
-  float* scores;       // [B][Hkv][max_pages]
-  int32_t* sel;        // [B][Hkv][K]
-  int32_t* sel_count;  // [B][Hkv]
-  int32_t* sel_phys;   // [B][Hkv][K] physical pages of the selection (nullable)
-  int32_t* status;
-  int Hkv, P, max_pages, K, s_pages, w_pages;
-  int ptab_in_smem;  // the sequence's page-table row is staged next to the keys
-};
 
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs a) {
   constexpr int NT = kSelectThreads;
-  using Bar = SelBar<-1, NT>;
   extern __shared__ uint32_t keys[];  // [max_pages] keys, then [max_pages] page table
   __shared__ uint32_t hist[kHistBins];
   __shared__ uint32_t misc[4], red[2 * (NT / 32)];
@@ -437,105 +67,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
   __shared__ int bin_page[kBinCap];
   __shared__ int warp_tot[NT / 32 + 1];
   const SelScratch sh{hist, bin_key, bin_page, warp_tot, red, misc};
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.x, b = blockIdx.y;
-  // The scoring grid passed its own wait before letting this grid start, so the
-  // inputs of the call (everything but the scores) are complete here.
-  const int L = min(max(a.seq_lens[b], 0), a.max_pages * a.P);
-  const int nb = (L + a.P - 1) / a.P;
-  const int32_t* ptab_g = a.page_table + (size_t)b * a.max_pages;
-  float* srow = a.scores + ((size_t)b * a.Hkv + h) * a.max_pages;
-  // 1. wait for the scores (one thread; the rest block on the CTA barrier)
-  if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
-  __syncthreads();
-  asm volatile("griddepcontrol.launch_dependents;");
-  int32_t* out = a.sel + ((size_t)b * a.Hkv + h) * a.K;
-  int32_t* cnt_out = a.sel_count + (size_t)b * a.Hkv + h;
-  int32_t* phys_out = a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.K : nullptr;
-  const int K = a.K;
-  if (nb <= K) {  // everything fits the budget
-    for (int i = tid; i < K; i += NT) {
-      out[i] = i < nb ? i : -1;
-      if (phys_out) phys_out[i] = i < nb ? ptab_g[i] : -1;
-    }
-    if (tid == 0) *cnt_out = nb;
-    return;
-  }
-  int32_t* ptab_s = a.ptab_in_smem ? reinterpret_cast<int32_t*>(keys + a.max_pages) : nullptr;
-  // 2. keys (8 loads in flight per thread) and the candidates' key range
-  const int wbeg = nb - a.w_pages;
-  uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
-  for (int p0 = 0; p0 < nb; p0 += NT * 8) {
-    float v[8];
-    int pt[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int p = p0 + k * NT + tid;
-      v[k] = p < nb ? __ldcg(srow + p) : 0.f;
-      pt[k] = (ptab_s && p < nb) ? ptab_g[p] : 0;
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int p = p0 + k * NT + tid;
-      if (p < nb) {
-        const float sv = v[k];
-        const bool forced = p < a.s_pages || p >= wbeg;
-        const uint32_t key = forced ? 0u : f32_order_key(sv);
-        keys[p] = key;
-        if (!forced) {
-          kmn = min(kmn, key);
-          kmx = max(kmx, key);
-        }
-        if (ptab_s) ptab_s[p] = pt[k];
-      }
-    }
-  }
-  block_key_range<NT, Bar>(kmn, kmx, red);
-
-  // 3. threshold: a candidate is taken when its key >= thr or it was marked kWin
-  const uint64_t thr = radix_select_threshold<NT, Bar>(keys, nb, a.s_pages, wbeg,
-                                                       K - a.s_pages - a.w_pages, kmn, kmx, sh);
-
-  // 4. ascending list: forced pages and taken candidates.  Each warp owns a contiguous
-  // run of pages (a multiple of 32) and compacts it with ballots; one block barrier
-  // gives every warp its offset.
-  auto taken = [&](int p) {
-    if (p < a.s_pages || p >= wbeg) return true;
-    const uint32_t key = keys[p];
-    return key == kWin || (uint64_t)key >= thr;
-  };
-  const int per_warp = ((nb + NT - 1) / NT) * 32;
-  const int w0 = min(nb, warp * per_warp), w1 = min(nb, w0 + per_warp);
-  int n_sel = 0;
-  for (int p0 = w0; p0 < w1; p0 += 32) {
-    const int p = p0 + lane;
-    n_sel += __popc(__ballot_sync(0xffffffffu, p < w1 && taken(p)));
-  }
-  if (lane == 0) warp_tot[warp] = n_sel;
-  __syncthreads();
-  int pos = 0, tot = 0;
-#pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    const int v = warp_tot[w];
-    pos += w < warp ? v : 0;
-    tot += v;
-  }
-  for (int p0 = w0; p0 < w1; p0 += 32) {
-    const int p = p0 + lane;
-    const bool tk = p < w1 && taken(p);
-    const unsigned m = __ballot_sync(0xffffffffu, tk);
-    if (tk) {
-      const int at = pos + __popc(m & ((1u << lane) - 1u));
-      out[at] = p;
-      if (phys_out) phys_out[at] = ptab_s ? ptab_s[p] : ptab_g[p];
-    }
-    pos += __popc(m);
-  }
-  for (int i = tot + tid; i < K; i += NT) {
-    out[i] = -1;
-    if (phys_out) phys_out[i] = -1;
-  }
-  if (tid == 0) *cnt_out = tot;
+  select_body<NT, SelBar<-1, NT>>(a, blockIdx.y, blockIdx.x, keys, sh);
 }
 
 static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem,
@@ -728,6 +260,237 @@ cudaError_t launch_score_select(const sa_geom& g, const void* q, void* summ, con
   if (e != cudaSuccess) return e;
   return launch_select(g, page_table, seq_lens, scores, K, sink_pages, window_pages, sel,
                        sel_count, sel_phys, status, stream);
+}
+
+// ---------------------------------------------------------------------------------------
+// Single-launch decode: the whole grouped-query step (scores with the newest pages'
+// refresh, the per-(sequence, KV head) selection, the gathered attention, the merge of
+// the cut pairs) in one persistent launch of one 288-thread CTA per SM, the CTAs all
+// resident (cooperative launch).  The phases run the same CTA programs as the separate
+// kernels; between them a grid barrier on a counter in the workspace header (zeroed
+// before the launch) hands the results over.  The barrier is bounded: a CTA that waits
+// longer than kWaitLimitNs reports SA_ERR_TIMEOUT and goes on.  The selection is spread
+// over the CTAs (CTA c takes pairs c, c + grid, ...) by its first 256 threads.
+// ---------------------------------------------------------------------------------------
+constexpr int kFusedThreads = kScoreThreads;  // 8 compute warps + 1 producer warp
+constexpr int kFusedSelectThreads = 256;
+static_assert(kFusedThreads == (kAttnWarps + 1) * 32, "phases share one CTA shape");
+
+// shared-memory scratch of the selection phase, carved after the keys (and page table)
+struct FusedSelLayout {
+  size_t keys, hist, bin_key, bin_page, warp_tot, red, misc, total;
+};
+__host__ __device__ inline FusedSelLayout fused_sel_layout(int max_pages, bool ptab) {
+  FusedSelLayout l;
+  size_t off = 0;
+  l.keys = off;
+  off += (size_t)(ptab ? 2 : 1) * max_pages * 4;
+  off = (off + 15) & ~size_t(15);
+  l.hist = off;
+  off += kHistBins * 4;
+  l.bin_key = off;
+  off += kBinCap * 4;
+  l.bin_page = off;
+  off += kBinCap * 4;
+  l.warp_tot = off;
+  off += (kFusedSelectThreads / 32 + 1) * 4;
+  l.red = off;
+  off += 2 * (kFusedSelectThreads / 32) * 4;
+  l.misc = off;
+  off += 4 * 4;
+  l.total = off;
+  return l;
+}
+
+// Grid barrier number `phase` (1, 2, ...) over the launch's CTAs; false after a timeout.
+__device__ __forceinline__ bool fused_grid_sync(int32_t* counter, int phase, int32_t* status) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's results are visible before it arrives
+    atomicAdd(counter, 1);
+    const int target = phase * (int)gridDim.x;
+    const uint64_t t0 = global_ns();
+    int ok = 1;
+    while (*(volatile int32_t*)counter < target) {
+      if (global_ns() - t0 > kWaitLimitNs) {
+        report(status, SA_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(200);
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+template <int D, int P, int SPW>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    fused_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap vmap, const ScoreArgs sa,
+                        const SelectArgs se, const AttnArgs at, const MergeArgs mg,
+                        int32_t* counter) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1. page scores (and the newest pages' refresh)
+  score_stream_body<D, false>(sa, smem_raw);
+  // the next phase's bulk copies land where this one read and wrote generically
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (!fused_grid_sync(counter, 1, sa.status)) return;
+  // 2. selections
+  {
+    const FusedSelLayout l = fused_sel_layout(se.max_pages, se.ptab_in_smem != 0);
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const SelScratch sh{reinterpret_cast<uint32_t*>(base + l.hist),
+                        reinterpret_cast<uint32_t*>(base + l.bin_key),
+                        reinterpret_cast<int*>(base + l.bin_page),
+                        reinterpret_cast<int*>(base + l.warp_tot),
+                        reinterpret_cast<uint32_t*>(base + l.red),
+                        reinterpret_cast<uint32_t*>(base + l.misc)};
+    using Bar = SelBar<3, kFusedSelectThreads>;
+    if (threadIdx.x < kFusedSelectThreads) {
+      for (int pr = blockIdx.x; pr < mg.n_pairs; pr += gridDim.x) {
+        select_body<kFusedSelectThreads, Bar>(se, pr / se.Hkv, pr % se.Hkv,
+                                              reinterpret_cast<uint32_t*>(base + l.keys), sh);
+        Bar::sync();  // the scratch is reused by the next pair
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (!fused_grid_sync(counter, 2, sa.status)) return;
+  // 3. attention over the selected pages
+  attend_gqa_body<D, P, kAttnWarps, SPW>(&kmap, &vmap, at, smem_raw);
+  if (!fused_grid_sync(counter, 3, sa.status)) return;
+  // 4. merge of the pairs cut by warp ranges: one warp per (pair, query head)
+  const int warp = threadIdx.x >> 5, n_warps = gridDim.x * (kFusedThreads / 32);
+  for (int wi = blockIdx.x * (kFusedThreads / 32) + warp; wi < mg.n_pairs * mg.G; wi += n_warps)
+    merge_task<D>(mg, wi, threadIdx.x & 31);
+}
+
+template <int D, int P>
+static cudaError_t launch_fused_t(const sa_geom& g, const FusedCall& f, cudaStream_t stream) {
+  constexpr int SPW = D <= 64 ? 4 : 3;
+  using S = AttnShape<D, P, kAttnWarps, SPW>;
+  const int n_cta = f.n_cta;
+  const int n_pairs = g.B * g.Hkv;
+  ScoreArgs sa = make_score_args(g, f.q, f.summ, f.page_table, f.seq_lens, f.scores, f.status,
+                                 false);
+  if (f.n_tail > 0) {
+    sa.k_cache = static_cast<const uint4*>(f.k_cache);
+    sa.summ_w = static_cast<uint4*>(f.summ);
+    sa.n_tail = f.n_tail < kMaxTail ? f.n_tail : kMaxTail;
+  }
+  SelectArgs se;
+  se.page_table = f.page_table;
+  se.seq_lens = f.seq_lens;
+  se.scores = f.scores;
+  se.sel = f.sel;
+  se.sel_count = f.sel_count;
+  se.sel_phys = f.sel_phys;
+  se.status = f.status;
+  se.Hkv = g.Hkv;
+  se.P = g.P;
+  se.max_pages = g.max_pages;
+  se.K = f.K;
+  se.s_pages = f.s_pages;
+  se.w_pages = f.w_pages;
+  const size_t score_b = score_smem(g, sa);
+  const size_t attn_b = S::smem_bytes(n_pairs);
+  se.ptab_in_smem = fused_sel_layout(g.max_pages, true).total + 128 <= score_b;
+  const size_t sel_b = fused_sel_layout(g.max_pages, se.ptab_in_smem != 0).total + 128;
+  size_t smem = score_b > attn_b ? score_b : attn_b;
+  if (sel_b > smem) smem = sel_b;
+  AttnArgs at;
+  at.q = static_cast<const uint16_t*>(f.q);
+  at.page_table = f.page_table;
+  at.seq_lens = f.seq_lens;
+  at.sel = f.sel;
+  at.sel_count = f.sel_count;
+  at.sel_phys = f.sel_phys;
+  at.part = f.part;
+  at.pre_out = f.pre;
+  at.out = f.out;
+  at.lse = f.lse;
+  at.status = f.status;
+  at.sel_stride = f.K;
+  at.Hq = g.Hq;
+  at.Hkv = g.Hkv;
+  at.B = g.B;
+  at.max_pages = g.max_pages;
+  at.n_pool = g.n_pool;
+  at.counts_from_lens = 1;
+  at.scale_log2 = f.scale * 1.4426950408889634f;
+  MergeArgs mg;
+  mg.part = f.part;
+  mg.pre = f.pre;
+  mg.out = f.out;
+  mg.lse = f.lse;
+  mg.n_pairs = n_pairs;
+  mg.G = g.Hq / g.Hkv;
+  mg.Hkv = g.Hkv;
+  mg.Hq = g.Hq;
+  mg.n_warps = n_cta * kAttnWarps;
+  CUtensorMap kmap, vmap;
+  const uint64_t rows = (uint64_t)g.n_pool * g.Hkv * P;
+  if (!encode_rows_tmap(&kmap, f.k_cache, D, rows, 64, S::CT)) return cudaErrorInvalidValue;
+  if (!encode_rows_tmap(&vmap, f.v_cache, D, rows, 64, S::CT)) return cudaErrorInvalidValue;
+  const void* kern = reinterpret_cast<const void*>(fused_decode_kernel<D, P, SPW>);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  int dev = 0, optin = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+      cudaSuccess)
+    return e;
+  if (smem + fa.sharedSizeBytes > (size_t)optin) return cudaErrorInvalidConfiguration;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+      cudaSuccess)
+    return e;
+  // every CTA must be resident at once for the grid barriers
+  int per_sm = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFusedThreads, smem)) !=
+      cudaSuccess)
+    return e;
+  if (per_sm < 1 || n_cta > per_sm * f.n_sm) return cudaErrorCooperativeLaunchTooLarge;
+  if ((e = cudaMemsetAsync(f.counter, 0, sizeof(int32_t), stream)) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_cta);
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int32_t* counter = f.counter;
+  void* args[] = {&kmap, &vmap, &sa, &se, &at, &mg, &counter};
+  return cudaLaunchKernelExC(&cfg, kern, args);
+}
+
+bool fused_supported(const sa_geom& g, int K, int n_sm) {
+  if (!(g.Dk == 64 || g.Dk == 128) || g.Dv != g.Dk || g.v_aliases_k) return false;
+  if (!(g.P == 16 || g.P == 32 || g.P == 64)) return false;
+  if (!score_supported(g)) return false;
+  // one CTA per SM covers the scoring slices and the attention ranges
+  return score_ctas(g, n_sm) <= n_sm && attend_ctas(g, K, n_sm) <= n_sm;
+}
+
+cudaError_t launch_fused(const sa_geom& g, const FusedCall& f, cudaStream_t stream) {
+#define SA_FUSED_CASE(DD, PP) \
+  if (g.Dk == DD && g.P == PP) return launch_fused_t<DD, PP>(g, f, stream);
+  SA_FUSED_CASE(64, 16)
+  SA_FUSED_CASE(64, 32)
+  SA_FUSED_CASE(64, 64)
+  SA_FUSED_CASE(128, 16)
+  SA_FUSED_CASE(128, 32)
+  SA_FUSED_CASE(128, 64)
+#undef SA_FUSED_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace sa
