@@ -13,7 +13,9 @@ step touches ~4.3 GB (> L2) and nothing is served from L2 across layers.
 The default llama32k run also times llama128k (131072 tokens per sequence), ragged
 (4 sequences of 64K-256K tokens, page 32) and mla (latent 576/512, 128 query heads) the
 same way over 8 layer pools each and adds their microseconds per layer-call and HBM
-fractions to the line's config (--no-extras skips them).  cpu_baseline is the CPU oracle
+fractions to the line's config, and every grouped-query run adds the same step as one
+persistent launch per layer (sa_sparse_decode_fused, single_launch_us_per_layer)
+(--no-extras skips them).  cpu_baseline is the CPU oracle
 on every host core (independent sequences on threads), its single-thread rate beside it.
 
 Metric: sparse-decode seq*heads/s = (sequence, query head) attention outputs of one
@@ -575,6 +577,38 @@ def run_native(args, rank, world, dist):
         cpu_v, cpu_done, cpu_t, cpu_cores = oracle_sample_mt(case, args.cpu_seconds, R, F8)
         cpu1 = oracle_sample(case, args.cpu_seconds / 2, R, F8)
     extras = {}
+    if world == 1 and args.extras and not g.v_aliases_k and R == 1 and not F8:
+        # the same step as one persistent launch per layer (sa_sparse_decode_fused), timed
+        # the headline's way on the headline's pools
+        def step_single():
+            for l in range(L_layers):
+                sa.sparse_decode_fused(g, qs[l], ks[l], vs[l], summs[l], pt, sl, case.budget,
+                                       case.sink, case.window, case.scale, ws, out=outs[l],
+                                       lse=lses[l], sel_out=sel, sel_count_out=cnt,
+                                       n_tail_refresh=1)
+        try:
+            with torch.cuda.stream(stream):
+                step_single()
+            torch.cuda.synchronize()
+            graph_f = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_f, stream=stream):
+                step_single()
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    graph_f.replay()
+                torch.cuda.synchronize()
+                f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                f0.record(stream)
+                for _ in range(args.steps):
+                    graph_f.replay()
+                f1.record(stream)
+            torch.cuda.synchronize()
+            assert ws.status() == sa.SA_OK
+            extras["single_launch_us_per_layer"] = (f0.elapsed_time(f1) * 1e3 /
+                                                    (args.steps * L_layers))
+            del graph_f
+        except sa.SaError:
+            extras["single_launch_us_per_layer"] = None
     if world == 1 and args.extras and args.workload == "llama32k" and R == 1 and not F8:
         # free the headline's pools first: the other configurations need the room
         del ks, vs, qs, summs, k0, v0, graph, graph_ev, graph_sc
