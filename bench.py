@@ -967,7 +967,9 @@ def run_prune(args, rank, world, dist):
 
 def recorded_traffic(kernel, workload):
     """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
-    there is none for this workload or the kernel's source changed since it was taken."""
+    there is none for this workload or the kernel's source changed since it was taken.
+    The source is hashed without its SA_TRACE_POINT lines, which expand to nothing
+    outside the traced build."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -978,7 +980,9 @@ def recorded_traffic(kernel, workload):
         return None
     src = os.path.join(ROOT, "paged_kv_cache_sa_b200", "csrc", rec["source"])
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        text = open(src, "rb").read().decode()
+        text = "".join(l for l in text.splitlines(True) if "SA_TRACE_POINT" not in l)
+        sha = hashlib.sha256(text.encode()).hexdigest()
     except OSError:
         return None
     return rec["dram_bytes_per_launch"] if sha == rec["source_sha256"] else None

@@ -288,8 +288,10 @@ int sa_sparse_decode_noalloc(const sa_geom* g, const void* q, const void* k_cach
  * of each entry as written by sa_select_pages; passing it also states that the
  * selection was made by sa_select_pages for these seq_lens with budget
  * sel_stride * P, so that sel_count[b][h] == min(ceil(seq_lens[b] / P), sel_stride)
- * (the kernel then derives the counts from seq_lens and starts earlier).  Without
- * sel_phys the page table and sel_count are read. */
+ * (the kernel then derives the counts from seq_lens and starts earlier; it reads
+ * seq_lens before the previous kernel of the stream has finished, so seq_lens must be
+ * unchanged since that selection).  Without sel_phys the page table and sel_count
+ * are read. */
 int sa_attend_selected(const sa_geom* g, const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* page_table, const int32_t* seq_lens, const int32_t* sel,
                        const int32_t* sel_count, const int32_t* sel_phys, int sel_stride,

@@ -42,17 +42,21 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    """Compile every csrc/*.cu and link lib/libsa.so; returns the library path."""
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra_flags=(), trace: bool = False) -> str:
+    """Compile every csrc/*.cu and link lib/libsa.so; returns the library path.  trace:
+    the same sources with -DSA_TRACE (phase-timeline points, include/sa_trace.h) into
+    lib/libsa_trace.so instead."""
+    objdir = OBJDIR + ("_trace" if trace else "")
+    lib = os.path.join(LIBDIR, "libsa_trace.so") if trace else LIB
+    os.makedirs(objdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
                      + glob.glob(os.path.join(INCLUDE, "*.h")))
     nv = nvcc()
-    flags = NVCC_FLAGS + list(extra_flags)
+    flags = NVCC_FLAGS + list(extra_flags) + (["-DSA_TRACE"] if trace else [])
 
     def compile_one(src):
-        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         if force or _stale(obj, [src, __file__] + headers):
             cmd = [nv] + ARCH + flags + ["-c", src, "-o", obj]
             if verbose:
@@ -66,15 +70,15 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or _stale(LIB, objs):
-        tmp = LIB + ".tmp.%d" % os.getpid()
+    if force or _stale(lib, objs):
+        tmp = lib + ".tmp.%d" % os.getpid()
         cmd = [nv] + ARCH + ["-shared", "-o", tmp] + objs + ["-Xcompiler", "-fPIC"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv))

@@ -47,8 +47,10 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
 template <int D>
 __global__ void __launch_bounds__(128) attend_merge_kernel(const MergeArgs a) {
   // one thread waits for the attention grid; the rest block on the CTA barrier
+  if (threadIdx.x == 0) SA_TRACE_POINT(3, 0);  // entry
   if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
+  if (threadIdx.x == 0) SA_TRACE_POINT(3, 1);  // attention visible
   asm volatile("griddepcontrol.launch_dependents;");
   const int wi = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (wi < a.n_pairs * a.G) merge_task<D>(a, wi, threadIdx.x & 31);
@@ -173,5 +175,9 @@ cudaError_t launch_attend(const sa_geom& g, const AttendCall& c, cudaStream_t st
 #undef SA_ATTEND_CASE
   return cudaErrorInvalidValue;
 }
+
+#ifdef SA_TRACE
+void trace_set_attend(void* buf) { cudaMemcpyToSymbol(sa_trace_buf, &buf, sizeof(buf)); }
+#endif
 
 }  // namespace sa

@@ -106,6 +106,7 @@ __device__ __forceinline__ void attend_gqa_body(const CUtensorMap* kmap, const C
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, n_cta = gridDim.x;
+  if (tid == 0) SA_TRACE_POINT(2, 0);  // entry
 
   if (tid == 0) {
     for (int s = 0; s < S::NST; ++s) {
@@ -171,7 +172,9 @@ __device__ __forceinline__ void attend_gqa_body(const CUtensorMap* kmap, const C
       }
     }
     // 3. the selection itself comes from the previous kernel of the stream
+    if (lane == 0) SA_TRACE_POINT(2, 1);  // lengths-only tables built
     if (a.counts_from_lens) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (lane == 0) SA_TRACE_POINT(2, 2);  // selection visible
     asm volatile("griddepcontrol.launch_dependents;");
     if (c == 0)
       for (int p = lane; p <= n_pairs; p += 32) a.pre_out[p] = pre[p];
@@ -207,6 +210,7 @@ __device__ __forceinline__ void attend_gqa_body(const CUtensorMap* kmap, const C
         u_nv[j] = nv;
       }
     }
+    if (lane == 0) SA_TRACE_POINT(2, 13);  // unit loads landed
     if (lane == 0) {
       sh_nu = nu;
       sh_U0 = U0;
@@ -214,6 +218,7 @@ __device__ __forceinline__ void attend_gqa_body(const CUtensorMap* kmap, const C
     }
     __syncwarp();
     named_bar(1, kThreads);  // tables ready
+    if (lane == 0) SA_TRACE_POINT(2, 3);  // unit tables ready
 
     // ===================== producer warp: TMA issue =====================
     if (lane == 0) {
@@ -371,6 +376,7 @@ __device__ __forceinline__ void attend_gqa_body(const CUtensorMap* kmap, const C
         atomicExch(&abort_flag, 1);
         ok = false;
       }
+      if (kc == 0 && lane == 0 && warp == 0) SA_TRACE_POINT(2, 4);  // first unit
       const int nv = ok ? u_nv[j] : 0;
       const uint32_t kbase = stage0 + st * S::STAGE_BYTES;
       const uint32_t vbase = kbase + S::KV_BYTES;
@@ -442,6 +448,7 @@ __device__ __forceinline__ void attend_gqa_body(const CUtensorMap* kmap, const C
       if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
     if (cur >= 0) finish(cur);
+    if (lane == 0) SA_TRACE_POINT(2, 5 + warp);  // warp's range done
   }
   __syncthreads();
   if (abort_flag && warp == NC && lane == 0) {

@@ -423,6 +423,14 @@ SA_EXPORT int sa_sparse_decode_fused(const sa_geom* g, const void* q, const void
   return cuda_status(e);
 }
 
+#ifdef SA_TRACE
+SA_EXPORT int sa_trace_set(void* device_buf) {
+  trace_set_score(device_buf);
+  trace_set_attend(device_buf);
+  return cuda_status(cudaGetLastError());
+}
+#endif
+
 // ---- fp8 summaries rounded outward (grouped-query geometry) ---------------------------
 
 SA_EXPORT size_t sa_summary_fp8_record_bytes(const sa_geom* g) {

@@ -34,6 +34,23 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Phase timeline (compiled in only with -DSA_TRACE, the build behind include/sa_trace.h):
+// SA_TRACE_POINT(kernel, event) stores %globaltimer at [kernel][CTA][event] of the buffer
+// that sa_trace_set installed (1024 CTA rows of 16 events per kernel).  The default build
+// expands it to nothing.
+#ifdef SA_TRACE
+static __device__ unsigned long long* sa_trace_buf = nullptr;
+__device__ __forceinline__ void sa_trace_point(int kid, int ev) {
+  if (sa_trace_buf) {
+    const size_t cta = blockIdx.x + (size_t)blockIdx.y * gridDim.x;
+    if (cta < 1024) sa_trace_buf[((size_t)kid * 1024 + cta) * 16 + ev] = global_ns();
+  }
+}
+#define SA_TRACE_POINT(kid, ev) ::sa::sa_trace_point(kid, ev)
+#else
+#define SA_TRACE_POINT(kid, ev) ((void)0)
+#endif
+
 // ------------------------------------------------------------------------------------
 // bf16 min/max with a total order (-0 < +0) via the signed-16-bit key
 // key(x) = x ^ (sign(x) ? 0x7FFF : 0); the map is its own inverse.

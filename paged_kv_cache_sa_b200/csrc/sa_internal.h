@@ -21,6 +21,12 @@ struct DecodePlan {
 
 bool make_decode_plan(const sa_geom& g, int budget, DecodePlan* plan);
 
+#ifdef SA_TRACE
+// the traced build: install the timeline buffer in each translation unit with trace points
+void trace_set_score(void* buf);
+void trace_set_attend(void* buf);
+#endif
+
 // ---- launchers (return the CUDA error of the launch) ----------------------------------
 cudaError_t launch_summaries(const sa_geom& g, const void* k_cache, const int32_t* page_table,
                              const int32_t* seq_lens, void* summ, int n_tail,

@@ -336,6 +336,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   // 1. page scores (and the newest pages' refresh)
   score_stream_body<D, false>(sa, smem_raw);
+  if (threadIdx.x == 0) SA_TRACE_POINT(4, 0);  // phase 1 done
   // the next phase's bulk copies land where this one read and wrote generically
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (!fused_grid_sync(counter, 1, sa.status)) return;
@@ -360,10 +361,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (threadIdx.x == 0) SA_TRACE_POINT(4, 1);  // phase 2 done
   if (!fused_grid_sync(counter, 2, sa.status)) return;
+  if (threadIdx.x == 0) SA_TRACE_POINT(4, 2);  // barrier 2 passed
   // 3. attention over the selected pages
   attend_gqa_body<D, P, kAttnWarps, SPW>(&kmap, &vmap, at, smem_raw);
+  if (threadIdx.x == 0) SA_TRACE_POINT(4, 3);  // phase 3 done
   if (!fused_grid_sync(counter, 3, sa.status)) return;
+  if (threadIdx.x == 0) SA_TRACE_POINT(4, 4);  // barrier 3 passed
   // 4. merge of the pairs cut by warp ranges: one warp per (pair, query head)
   const int warp = threadIdx.x >> 5, n_warps = gridDim.x * (kFusedThreads / 32);
   for (int wi = blockIdx.x * (kFusedThreads / 32) + warp; wi < mg.n_pairs * mg.G; wi += n_warps)
@@ -492,5 +497,9 @@ cudaError_t launch_fused(const sa_geom& g, const FusedCall& f, cudaStream_t stre
 #undef SA_FUSED_CASE
   return cudaErrorInvalidValue;
 }
+
+#ifdef SA_TRACE
+void trace_set_score(void* buf) { cudaMemcpyToSymbol(sa_trace_buf, &buf, sizeof(buf)); }
+#endif
 
 }  // namespace sa

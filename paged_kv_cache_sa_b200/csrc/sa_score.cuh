@@ -153,6 +153,7 @@ __device__ __forceinline__ void score_stream_body(const ScoreArgs& a, uint8_t* s
   __shared__ int abort_flag;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, n_cta = gridDim.x;
+  if (tid == 0) SA_TRACE_POINT(0, 0);  // entry
 
   if (tid == 0) {
     for (int s = 0; s < a.NST; ++s) {
@@ -169,6 +170,7 @@ __device__ __forceinline__ void score_stream_body(const ScoreArgs& a, uint8_t* s
   // per SM, contending); launched as this grid exits, they spread over idle SMs.
   if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
+  if (tid == 0) SA_TRACE_POINT(0, 1);  // dependency wait passed
 
   // The slice of the flattened tile list this CTA streams: every warp derives it from
   // the sequence lengths itself, so no CTA-wide barrier stands before the first copy.
@@ -202,6 +204,7 @@ __device__ __forceinline__ void score_stream_body(const ScoreArgs& a, uint8_t* s
     }
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
     __syncwarp();
+    if (lane == 0) SA_TRACE_POINT(0, 2);  // slice tables ready
 
     // 2. bulk-copy issue: lanes 0-15 check and copy one page each, lane 16 the queries
     const uint32_t slot_data = (uint32_t)a.HG * a.rec_bytes;  // one page's records of the group
@@ -288,6 +291,7 @@ __device__ __forceinline__ void score_stream_body(const ScoreArgs& a, uint8_t* s
         atomicExch(&abort_flag, 1);
         ok = false;
       }
+      if (ok && k == grp && lane == 0 && warp == 0) SA_TRACE_POINT(0, 3);  // first stage
       if (ok) {
         const int b = t_b[k], h = t_hg[k] * a.HG + hh, p0 = t_p0[k], np = t_np[k];
         const int vm = t_vm[k];
@@ -354,6 +358,7 @@ __device__ __forceinline__ void score_stream_body(const ScoreArgs& a, uint8_t* s
       if (lane == 0) mbar_arrive(&empty_bar[s]);
     }
   }
+  if (lane == 0 && warp == 0) SA_TRACE_POINT(0, 4);  // consumer 0 done
   if (warp == kScoreConsumers) {
     // scores past each sequence's last page are -inf (pairs spread over the CTAs)
     for (int pr = c; pr < a.B * a.Hkv; pr += n_cta) {
@@ -403,6 +408,7 @@ __device__ __forceinline__ void select_body(const SelectArgs& a, int b, int h, u
   if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   Bar::sync();
   asm volatile("griddepcontrol.launch_dependents;");
+  if (tid == 0) SA_TRACE_POINT(1, 0);  // scores visible
   int32_t* out = a.sel + ((size_t)b * a.Hkv + h) * a.K;
   int32_t* cnt_out = a.sel_count + (size_t)b * a.Hkv + h;
   int32_t* phys_out = a.sel_phys ? a.sel_phys + ((size_t)b * a.Hkv + h) * a.K : nullptr;
@@ -444,11 +450,14 @@ __device__ __forceinline__ void select_body(const SelectArgs& a, int b, int h, u
       }
     }
   }
+  if (tid == 0) SA_TRACE_POINT(1, 4);  // this thread's keys stored
   block_key_range<NT, Bar>(kmn, kmx, red);
+  if (tid == 0) SA_TRACE_POINT(1, 1);  // keys and their range
 
   // 3. threshold: a candidate is taken when its key >= thr or it was marked kWin
   const uint64_t thr = radix_select_threshold<NT, Bar>(keys, nb, a.s_pages, wbeg,
                                                        K - a.s_pages - a.w_pages, kmn, kmx, sh);
+  if (tid == 0) SA_TRACE_POINT(1, 2);  // threshold
 
   // 4. ascending list: forced pages and taken candidates.  Each warp owns a contiguous
   // run of pages (a multiple of 32) and compacts it with ballots; one block barrier
@@ -467,6 +476,7 @@ __device__ __forceinline__ void select_body(const SelectArgs& a, int b, int h, u
   }
   if (lane == 0) warp_tot[warp] = n_sel;
   Bar::sync();
+  if (tid == 0) SA_TRACE_POINT(1, 7);  // list counts
   int pos = 0, tot = 0;
 #pragma unroll
   for (int w = 0; w < NT / 32; ++w) {
@@ -490,6 +500,7 @@ __device__ __forceinline__ void select_body(const SelectArgs& a, int b, int h, u
     if (phys_out) phys_out[i] = -1;
   }
   if (tid == 0) *cnt_out = tot;
+  if (tid == 0) SA_TRACE_POINT(1, 3);  // list written
 }
 
 }  // namespace sa

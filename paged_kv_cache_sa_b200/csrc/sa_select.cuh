@@ -229,6 +229,7 @@ __device__ uint64_t radix_select_threshold(uint32_t* keys, int nb, int s_pages, 
         atomicAdd(&sh.hist[(key >> lo) & dmask], 1u);
     }
     Bar::sync();
+    if (tid == 0) SA_TRACE_POINT(1, 5);  // histogram built
     // bins owned BPT per thread; candidates in bins above each thread's range
     constexpr int BPT = kHistBins / NT;
     int mine = 0;
@@ -246,6 +247,7 @@ __device__ uint64_t radix_select_threshold(uint32_t* keys, int nb, int s_pages, 
       run += cnt;
     }
     Bar::sync();
+    if (tid == 0) SA_TRACE_POINT(1, 6);  // boundary bin found
     const uint32_t bstar = sh.misc[0];
     k_need -= (int)sh.misc[1];
     const int nbin = sh.hist[bstar];

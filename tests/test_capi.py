@@ -1,5 +1,6 @@
 """The C-ABI library builds, loads without a GPU, and exports exactly what
-include/sa.h declares; the CPU-only host logic of the binding."""
+include/sa.h declares (the traced build: sa.h and include/sa_trace.h); the CPU-only host
+logic of the binding."""
 
 import ctypes
 import os
@@ -11,21 +12,32 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared():
-    src = open(os.path.join(ROOT, "include", "sa.h")).read()
+def _declared(header="sa.h"):
+    src = open(os.path.join(ROOT, "include", header)).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", src)))
 
 
-@pytest.fixture(scope="module")
-def libpath():
+def _build(**kw):
     # build.py by path: importing the package first would load a possibly stale library
     import importlib.util
     spec = importlib.util.spec_from_file_location(
         "_sa_build", os.path.join(ROOT, "paged_kv_cache_sa_b200", "build.py"))
     b = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(b)
-    return b.build()
+    return b.build(**kw)
+
+
+def _exported(path):
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True,
+                         text=True).stdout
+    return sorted({ln.split()[-1] for ln in out.splitlines()
+                   if ln.split() and ln.split()[-1].startswith("sa_")})
+
+
+@pytest.fixture(scope="module")
+def libpath():
+    return _build()
 
 
 def test_header_declares_the_expected_entry_points():
@@ -44,11 +56,22 @@ def test_library_exports_every_declared_symbol(libpath):
     lib = ctypes.CDLL(libpath)
     for name in _declared():
         assert hasattr(lib, name), name
-    out = subprocess.run(["nm", "-D", "--defined-only", libpath], capture_output=True,
-                         text=True).stdout
-    exported = sorted({ln.split()[-1] for ln in out.splitlines()
-                       if ln.split() and ln.split()[-1].startswith("sa_")})
-    assert exported == _declared()
+    assert _exported(libpath) == _declared()
+
+
+def test_every_header_is_covered():
+    assert sorted(os.listdir(os.path.join(ROOT, "include"))) == ["sa.h", "sa_trace.h"]
+
+
+def test_traced_library_exports_sa_h_and_sa_trace_h():
+    """The phase-timeline build: everything libsa.so exports plus sa_trace_set."""
+    path = _build(trace=True)
+    lib = ctypes.CDLL(path)
+    want = sorted(set(_declared()) | set(_declared("sa_trace.h")))
+    assert _declared("sa_trace.h") == ["sa_trace_set"]
+    for name in want:
+        assert hasattr(lib, name), name
+    assert _exported(path) == want
 
 
 def test_binding_loads_and_sizes_workspaces(libpath):
