@@ -422,34 +422,40 @@ __device__ __forceinline__ void select_body(const SelectArgs& a, int b, int h, u
     return;
   }
   int32_t* ptab_s = a.ptab_in_smem ? reinterpret_cast<int32_t*>(keys + a.max_pages) : nullptr;
-  // 2. keys (8 loads in flight per thread) and the candidates' key range
+  // 2. keys (8 loads in flight per thread) and the candidates' key range.  The
+  //    page-table row goes to shared memory by asynchronous copies (no registers held),
+  //    waited for before the list is written.
   const int wbeg = nb - a.w_pages;
   uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
   for (int p0 = 0; p0 < nb; p0 += NT * 8) {
     float v[8];
-    int pt[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int p = p0 + k * NT + tid;
       v[k] = p < nb ? __ldcg(srow + p) : 0.f;
-      pt[k] = (ptab_s && p < nb) ? ptab_g[p] : 0;
+    }
+    if (ptab_s) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int p = p0 + k * NT + tid;
+        if (p < nb) cp_async4(ptab_s + p, ptab_g + p);
+      }
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int p = p0 + k * NT + tid;
       if (p < nb) {
-        const float sv = v[k];
         const bool forced = p < a.s_pages || p >= wbeg;
-        const uint32_t key = forced ? 0u : f32_order_key(sv);
+        const uint32_t key = forced ? 0u : f32_order_key(v[k]);
         keys[p] = key;
         if (!forced) {
           kmn = min(kmn, key);
           kmx = max(kmx, key);
         }
-        if (ptab_s) ptab_s[p] = pt[k];
       }
     }
   }
+  asm volatile("cp.async.commit_group;" ::: "memory");
   if (tid == 0) SA_TRACE_POINT(1, 4);  // this thread's keys stored
   block_key_range<NT, Bar>(kmn, kmx, red);
   if (tid == 0) SA_TRACE_POINT(1, 1);  // keys and their range
@@ -475,6 +481,7 @@ __device__ __forceinline__ void select_body(const SelectArgs& a, int b, int h, u
     n_sel += __popc(__ballot_sync(0xffffffffu, p < w1 && taken(p)));
   }
   if (lane == 0) warp_tot[warp] = n_sel;
+  asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's page-table copies
   Bar::sync();
   if (tid == 0) SA_TRACE_POINT(1, 7);  // list counts
   int pos = 0, tot = 0;

@@ -269,15 +269,18 @@ __device__ uint64_t radix_select_threshold(uint32_t* keys, int nb, int s_pages, 
         }
       }
       Bar::sync();
-      if (tid < nbin) {
-        const uint32_t key = sh.bin_key[tid];
-        const int pg = sh.bin_page[tid];
+      // each warp ranks members w, w + NT / 32, ...; its lanes split the comparisons
+      const int lane = tid & 31;
+      for (int i = tid >> 5; i < nbin; i += NT / 32) {
+        const uint32_t key = sh.bin_key[i];
+        const int pg = sh.bin_page[i];
         int rank = 0;
-        for (int j = 0; j < nbin; ++j) {
+        for (int j = lane; j < nbin; j += 32) {
           const uint32_t kj = sh.bin_key[j];
           rank += kj > key || (kj == key && sh.bin_page[j] < pg);
         }
-        if (rank < k_need) keys[pg] = kWin;
+        rank = __reduce_add_sync(0xffffffffu, rank);
+        if (lane == 0 && rank < k_need) keys[pg] = kWin;
       }
       thr = (uint64_t)pval + (1ull << lo);
       state = 1;
