@@ -262,9 +262,8 @@ int sa_sparse_decode_fp8(const sa_geom* g, const void* q, const void* k_cache,
  *    call before any stream capture.  The address is cached per device for the life of
  *    the process: resetting a device (cudaDeviceReset) is not supported afterwards.
  *  - Zeroing: the module's load zero-fills the scratch.  Every call clears the status
- *    word on `stream` before its first launch; the rest of the header (the single-launch
- *    decode's cursor, CTA count and call tag) must carry over from call to call and is
- *    kept consistent by the kernels themselves.
+ *    word on `stream` before its first launch; the rest of the scratch is written by
+ *    each call before it is read, as in a workspace, so nothing else carries over.
  *  - status_out (nullable, device int32): receives, on `stream`, the bit-OR of the
  *    device-detected errors of this call ((1 << -status) per error, 0 when none).  With
  *    status_out NULL those errors are dropped: the next call clears the word, and no
