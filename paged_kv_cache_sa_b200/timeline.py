@@ -42,7 +42,9 @@ KERNELS = ["scoring", "selection", "attention", "merge", "single launch"]
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--workload", default="llama32k")
+    # the grouped-query workloads: the latent geometry's kernels carry no trace points
+    ap.add_argument("--workload", default="llama32k",
+                    choices=["tiny", "llama32k", "llama128k", "ragged"])
     ap.add_argument("--fused", action="store_true", help="time sa_sparse_decode_fused")
     args = ap.parse_args()
 
