@@ -134,41 +134,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// try_wait that lets the hardware suspend the thread until the phase completes (or
-// `hint_ns` passes), instead of returning at once: waiting warps then issue nothing.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
-                                                   uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait built on suspending try_waits (each suspends for at most 1 ms).
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait_hint(bar, parity, 1000000u)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    if (mbar_try_wait_hint(bar, parity, 1000000u)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-
-// 2-D tiled TMA load global -> shared, completion counted on `bar` (no multicast).
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
-                                            int32_t y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Untiled bulk copy global -> shared (no multicast): both addresses and `bytes` are
 // multiples of 16; completion counted on `bar`.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
@@ -189,7 +154,8 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
   return pol;
 }
 
-// tma_load_2d with an L2 cache policy.
+// 2-D tiled TMA load global -> shared (no multicast) with an L2 cache policy;
+// completion counted on `bar`.
 __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map,
                                                  int32_t x, int32_t y, uint64_t* bar,
                                                  uint64_t policy) {
