@@ -1,5 +1,6 @@
-"""Host-side pieces of bench.py: the algorithmic byte count per layer-call (bf16 and fp8
-summaries) and the oracle's timed sample, on CPU."""
+"""Host-side pieces of bench.py, on CPU: the algorithmic byte count per layer-call (bf16
+and fp8 summaries), the oracle's timed sample, and the lookup of the committed DRAM
+traffic records."""
 
 import os
 import sys
@@ -37,3 +38,29 @@ def test_oracle_sample_both_formats_and_reuse():
         for r in (1, 3):
             v, done, t = bench.oracle_sample(case, 0.05, select_every=r, fp8=fp8)
             assert done >= 1 and t > 0 and v > 0
+
+
+def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu record only while the kernel's source
+    is the one measured; SA_TRACE_POINT lines (nothing outside the traced build) do not
+    count as a change."""
+    import hashlib
+    import json
+    src_dir = tmp_path / "paged_kv_cache_sa_b200" / "csrc"
+    src_dir.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    body = "int a;\nint b;\n"
+    sha = hashlib.sha256(body.encode()).hexdigest()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({
+        "k": {"workload": "llama32k", "source": "x.cuh", "source_sha256": sha,
+              "dram_bytes_per_launch": 1234}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    src = src_dir / "x.cuh"
+    src.write_text(body)
+    assert bench.recorded_traffic("k", "llama32k") == 1234
+    assert bench.recorded_traffic("k", "llama128k") is None      # another workload
+    assert bench.recorded_traffic("other", "llama32k") is None   # no record
+    src.write_text("int a;\n  SA_TRACE_POINT(0, 1);  // stamp\nint b;\n")
+    assert bench.recorded_traffic("k", "llama32k") == 1234
+    src.write_text("int a;\nint c;\n")
+    assert bench.recorded_traffic("k", "llama32k") is None       # the kernel changed
