@@ -290,6 +290,36 @@ def workload_config(case, args, layers):
     }
 
 
+def selection_counts(case):
+    """Pages every (sequence, KV head) selects: min(ceil(len / P), budget / P), as the
+    library's selection does by construction."""
+    g = case.geom
+    nb = (np.asarray(case.seq_lens, dtype=np.int64) + g.P - 1) // g.P
+    k = np.minimum(nb, case.budget // g.P).astype(np.int32)
+    return np.repeat(k[:, None], g.Hkv, axis=1)
+
+
+def step_bytes_of(case, args, layers, sel_count):
+    """Algorithmic bytes of one step: attention every layer, scoring and selection (with
+    the newest pages' refresh) every select_every layers."""
+    sel_b, att_b, upd_b = layer_bytes(case.geom, case.seq_lens, sel_count, case.geom.P,
+                                      args.summaries == "fp8")
+    R = args.select_every
+    return layers * att_b + ((layers + R - 1) // R) * (sel_b + upd_b)
+
+
+def run_config(case, args, layers, world, step_bytes):
+    """workload_config plus the run's L2 and parallelism description, worded as the
+    native line words them."""
+    return {
+        **workload_config(case, args, layers),
+        "l2": "inputs larger than L2: %d distinct layer pools, %.2f GB touched per step"
+              % (layers, step_bytes / 1e9),
+        "parallelism": "replicas (batch split), no collective" if world > 1 else "1 GPU",
+        "algorithmic_bytes_per_layer": step_bytes / layers,
+    }
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -316,7 +346,8 @@ def run_reference(args, rank, world):
         "unit": "seq*heads/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "ms_per_step": None,
-        "config": workload_config(case, args, args.layers),
+        "config": run_config(case, args, args.layers, world,
+                             step_bytes_of(case, args, args.layers, selection_counts(case))),
         "cpu_baseline": {"value": v, "unit": "seq*heads/s", "cores": cores, "kind": "oracle",
                          "sample": "%d (sequence, layer) decode calls of layer 0 "
                                    "(score+select%s, attend; all %d heads) on %d host "

@@ -64,3 +64,25 @@ def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     assert bench.recorded_traffic("k", "llama32k") == 1234
     src.write_text("int a;\nint c;\n")
     assert bench.recorded_traffic("k", "llama32k") is None       # the kernel changed
+
+
+def test_reference_arm_config_matches_the_native_line():
+    """The reference arm describes the workload with the native line's static keys: the
+    same L2 and parallelism wording and the same algorithmic bytes (llama32k, 32 layers:
+    134,841,344 B per layer-call, the figure the native bench prints from its measured
+    selection counts)."""
+    import argparse
+    case = synth.decode_case("llama32k")
+    args = argparse.Namespace(workload="llama32k", summaries="bf16", select_every=1)
+    cnt = bench.selection_counts(case)
+    assert cnt.shape == (case.geom.B, case.geom.Hkv)
+    assert (cnt == case.budget // case.geom.P).all()
+    sb = bench.step_bytes_of(case, args, 32, cnt)
+    cfg = bench.run_config(case, args, 32, 1, sb)
+    assert cfg["algorithmic_bytes_per_layer"] == 134841344
+    assert cfg["l2"] == "inputs larger than L2: 32 distinct layer pools, 4.31 GB touched per step"
+    assert cfg["parallelism"] == "1 GPU"
+    assert bench.run_config(case, args, 32, 2, sb)["parallelism"].startswith("replicas")
+    # short sequences select all their pages
+    short = synth.decode_case("tiny", B=2, seq_lens=[4096, 100], Hkv=1, Hq=4)
+    assert bench.selection_counts(short).tolist() == [[short.budget // 16], [7]]
